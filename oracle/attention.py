@@ -1,0 +1,302 @@
+"""Exact scaled-dot-product attention and its gradient in plain fp64 NumPy (the oracle).
+
+TEST INFRASTRUCTURE ONLY (see the package docstring): never imported by the product path.
+
+What is computed, and where it is defined:
+
+* Forward. "Breaking the Memory Wall: A Deep Dive into FlashAttention" (codethepapers.com),
+  section "The Problem: The Memory Wall": P = softmax(Q K^T / sqrt(d)) and the output is the
+  P-weighted sum of V rows; section "The Incremental Softmax Trick" gives
+  softmax(x_i) = e^{x_i} / sum_j e^{x_j}. The three pages agree that the method is exact
+  ("How FlashAttention Actually Works", section "Practical Takeaways": mathematically identical
+  to standard attention), so the oracle is the unchunked definition, not the tiled algorithm.
+  Per row i, with s_ij = scale * q_i . k_j:
+      m_i   = max_j s_ij                       (running maximum m, "The Secret Weapon: Online
+      l_i   = sum_j exp(s_ij - m_i)             Softmax", same page, names m and l)
+      O_i   = sum_j exp(s_ij - m_i) v_j / l_i
+      lse_i = m_i + ln l_i                      (natural log; the stored "normalization
+                                                 factors" of "Backward Pass Recomputation")
+  The max subtraction changes nothing mathematically; it keeps exp() in range.
+* Causal masking (key j visible to query i iff j <= i, square, top-left aligned): masked
+  entries are left out of every sum, i.e. they contribute exactly zero. The pages name masking
+  only as one of standard attention's HBM passes ("The GPU Memory Wall: HBM vs. SRAM").
+* Backward. The pages say only that the scores are recomputed on chip and the gradients
+  calculated ("The Backward Pass: Recomputation"). The formulas are the calculus of the
+  definition above, with P_ij = exp(s_ij - lse_i) and L a scalar loss with dO = dL/dO:
+      dV = P^T dO
+      dP = dO V^T
+      D_i = sum_c dO_ic O_ic          (= sum_j P_ij dP_ij, the softmax-Jacobian row term)
+      dS = P o (dP - D)               (o = elementwise product; masked entries are exactly 0)
+      dQ = scale * dS K,   dK = scale * dS^T Q
+* Tiled forward with online softmax. "How does FlashAttention optimize memory and speed via
+  tiling?" (iloveeagents.com), section "Core Technical Innovations", item 2 gives the update
+      m^(2) = max(m^(1), m~),  d^(2) = e^{m^(1) - m^(2)} d^(1) + e^{m~ - m^(2)} d~
+  and "How FlashAttention Actually Works", section "How Tiling Works", gives the loop order
+  (blocks of K/V outside, blocks of Q inside). ``tiled_attention_forward`` follows those steps,
+  with the partial output rescaled by the same factor as the running sum; it is used only to
+  pin that the tiled algorithm reaches the definition for every block size.
+
+Inputs are the exact bf16 values sent to the GPU, widened to float64; ``scale`` is the fp32
+value passed to the kernels, widened to float64.
+
+Rows are processed in blocks of ``block_rows`` only to bound memory to O(block_rows * N); each
+row's arithmetic is the definition above and does not depend on the blocking (a test checks
+this).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "attention_probabilities",
+    "attention_forward",
+    "attention_backward",
+    "attention_rows",
+    "attention_keys",
+    "online_softmax_stats",
+    "tiled_attention_forward",
+]
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def _visible(i: int, n_keys: int, causal: bool) -> int:
+    """Number of keys visible to query row i (keys 0 .. result-1)."""
+    return min(i + 1, n_keys) if causal else n_keys
+
+
+def _head_iter(shape):
+    """Iterate over every leading index of a [..., N, d] array."""
+    lead = shape[:-2]
+    return np.ndindex(*lead) if lead else iter([()])
+
+
+def _softmax_block(s: np.ndarray, mask: np.ndarray | None):
+    """Row statistics of a block of scores s [r, n] with optional visibility mask.
+
+    Returns (m, e, l): row max over visible entries, e = exp(s - m) with masked entries set to
+    exactly 0, and l = row sum of e.
+    """
+    if mask is None:
+        m = s.max(axis=1)
+        e = np.exp(s - m[:, None])
+    else:
+        m = np.where(mask, s, -np.inf).max(axis=1)
+        e = np.where(mask, np.exp(np.where(mask, s, 0.0) - m[:, None]), 0.0)
+    return m, e, e.sum(axis=1)
+
+
+def _causal_mask(r0: int, r1: int, n_keys: int) -> np.ndarray:
+    rows = np.arange(r0, r1)[:, None]
+    cols = np.arange(n_keys)[None, :]
+    return cols <= rows
+
+
+def attention_probabilities(q, k, scale: float, causal: bool = False) -> np.ndarray:
+    """P = softmax(scale * Q K^T) per the definition (codethepapers.com, "The Problem: The
+    Memory Wall"), masked entries exactly 0. Shapes: q [..., N, d], k [..., M, d] ->
+    [..., N, M]. Small inputs only (materialises N x M)."""
+    q, k = _f64(q), _f64(k)
+    scale = float(np.float64(scale))
+    out = np.zeros(q.shape[:-1] + (k.shape[-2],), dtype=np.float64)
+    for idx in _head_iter(q.shape):
+        s = scale * (q[idx] @ k[idx].T)
+        mask = _causal_mask(0, q.shape[-2], k.shape[-2]) if causal else None
+        _, e, l = _softmax_block(s, mask)
+        out[idx] = e / l[:, None]
+    return out
+
+
+def attention_forward(q, k, v, scale: float, causal: bool = False, block_rows: int = 512):
+    """Exact attention forward: returns (O [..., N, d], lse [..., N]) in float64.
+
+    Definition: codethepapers.com, "The Problem: The Memory Wall" (P = softmax(QK^T/sqrt d),
+    output P V) with the running max m and sum l of hot.atechcom.net, "The Secret Weapon:
+    Online Softmax"; lse = m + ln l. Masked entries (causal, j > i) contribute exactly 0.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    scale = float(np.float64(scale))
+    n, nk = q.shape[-2], k.shape[-2]
+    o = np.zeros(q.shape[:-1] + (v.shape[-1],), dtype=np.float64)
+    lse = np.zeros(q.shape[:-1], dtype=np.float64)
+    for idx in _head_iter(q.shape):
+        qh, kh, vh = q[idx], k[idx], v[idx]
+        for r0 in range(0, n, block_rows):
+            r1 = min(n, r0 + block_rows)
+            # keys beyond the last visible one of this block are masked for every row in it
+            kv_end = _visible(r1 - 1, nk, causal)
+            s = scale * (qh[r0:r1] @ kh[:kv_end].T)
+            mask = _causal_mask(r0, r1, kv_end) if causal else None
+            m, e, l = _softmax_block(s, mask)
+            o[idx][r0:r1] = (e @ vh[:kv_end]) / l[:, None]
+            lse[idx][r0:r1] = m + np.log(l)
+    return o, lse
+
+
+def attention_backward(q, k, v, do, scale: float, causal: bool = False, block_rows: int = 512,
+                       return_forward: bool = False):
+    """Gradient of exact attention: returns (dQ, dK, dV) in float64 (and (O, lse) if asked).
+
+    Recomputes O and lse from the definition (attention_forward), then
+    P = exp(S - lse), dV = P^T dO, dP = dO V^T, D = rowsum(dO o O), dS = P o (dP - D),
+    dQ = scale dS K, dK = scale dS^T Q. These are the calculus of the forward definition; the
+    pages only state that scores are recomputed on chip in the backward ("How FlashAttention
+    Actually Works", "The Backward Pass: Recomputation"). D uses the oracle's own fp64 O.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    scale = float(np.float64(scale))
+    o, lse = attention_forward(q, k, v, scale, causal, block_rows)
+    n, nk = q.shape[-2], k.shape[-2]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for idx in _head_iter(q.shape):
+        qh, kh, vh, doh = q[idx], k[idx], v[idx], do[idx]
+        dd = np.sum(doh * o[idx], axis=1)  # D_i
+        for r0 in range(0, n, block_rows):
+            r1 = min(n, r0 + block_rows)
+            kv_end = _visible(r1 - 1, nk, causal)
+            s = scale * (qh[r0:r1] @ kh[:kv_end].T)
+            p = np.exp(s - lse[idx][r0:r1, None])
+            if causal:
+                p = np.where(_causal_mask(r0, r1, kv_end), p, 0.0)
+            dv[idx][:kv_end] += p.T @ doh[r0:r1]
+            dp = doh[r0:r1] @ vh[:kv_end].T
+            ds = p * (dp - dd[r0:r1, None])
+            dq[idx][r0:r1] = scale * (ds @ kh[:kv_end])
+            dk[idx][:kv_end] += scale * (ds.T @ qh[r0:r1])
+    if return_forward:
+        return dq, dk, dv, o, lse
+    return dq, dk, dv
+
+
+def attention_rows(q, k, v, scale: float, causal: bool, rows, do=None):
+    """Forward (and dQ) for selected query rows only; cost O(N d) per row.
+
+    rows: iterable of index tuples (leading indices..., i), e.g. (b, h, i) for [B, H, N, d].
+    Returns (O_rows [n, d], lse_rows [n]) or, with dO given, (O_rows, lse_rows, dQ_rows).
+    Each row follows the same definition as attention_forward / attention_backward.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    do = None if do is None else _f64(do)
+    scale = float(np.float64(scale))
+    rows = [tuple(int(t) for t in r) for r in rows]
+    nk = k.shape[-2]
+    o_out = np.zeros((len(rows), v.shape[-1]))
+    lse_out = np.zeros(len(rows))
+    dq_out = np.zeros((len(rows), q.shape[-1])) if do is not None else None
+    for t, r in enumerate(rows):
+        head, i = r[:-1], r[-1]
+        vis = _visible(i, nk, causal)
+        kh, vh = k[head][:vis], v[head][:vis]
+        s = scale * (kh @ q[head][i])
+        m = s.max()
+        e = np.exp(s - m)
+        l = e.sum()
+        o_i = (e @ vh) / l
+        o_out[t] = o_i
+        lse_out[t] = m + np.log(l)
+        if do is not None:
+            p = e / l
+            do_i = do[head][i]
+            dp = vh @ do_i
+            ds = p * (dp - do_i @ o_i)
+            dq_out[t] = scale * (ds @ kh)
+    if do is not None:
+        return o_out, lse_out, dq_out
+    return o_out, lse_out
+
+
+def attention_keys(q, k, v, do, scale: float, causal: bool, head, keys, block_rows: int = 512):
+    """dK and dV rows for selected keys j of one head (leading index tuple `head`).
+
+    dV_j = sum_i P_ij dO_i and dK_j = scale sum_i dS_ij q_i over the query rows that see key j.
+    Needs lse_i and D_i of every row of the head, so the head's full forward is computed first.
+    Returns (dK_rows [n, d], dV_rows [n, d]).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    scale = float(np.float64(scale))
+    head = tuple(int(t) for t in head)
+    qh, kh, vh, doh = q[head], k[head], v[head], do[head]
+    o, lse = attention_forward(qh, kh, vh, scale, causal, block_rows)
+    dd = np.sum(doh * o, axis=1)
+    n = qh.shape[0]
+    dk_out = np.zeros((len(keys), kh.shape[1]))
+    dv_out = np.zeros((len(keys), vh.shape[1]))
+    for t, j in enumerate(int(x) for x in keys):
+        i0 = j if causal else 0  # rows i >= j see key j under the causal mask
+        s = scale * (qh[i0:n] @ kh[j])
+        p = np.exp(s - lse[i0:n])
+        dv_out[t] = p @ doh[i0:n]
+        dp = doh[i0:n] @ vh[j]
+        ds = p * (dp - dd[i0:n])
+        dk_out[t] = scale * (ds @ qh[i0:n])
+    return dk_out, dv_out
+
+
+def online_softmax_stats(logits, block: int):
+    """Running (max, sum) of one row of logits processed in chunks of `block` entries.
+
+    The update is the one of iloveeagents.com, "Core Technical Innovations", item 2:
+    m^(2) = max(m^(1), m~) and d^(2) = e^{m^(1) - m^(2)} d^(1) + e^{m~ - m^(2)} d~, where m~ and
+    d~ are the chunk's own max and sum of e^{x - m~}. Returns (m, d) with d = sum_j e^{x_j - m}.
+    """
+    x = _f64(logits).reshape(-1)
+    m = -np.inf
+    d = 0.0
+    for c0 in range(0, x.size, block):
+        chunk = x[c0:c0 + block]
+        m_chunk = chunk.max()
+        d_chunk = np.exp(chunk - m_chunk).sum()
+        m_new = max(m, m_chunk)
+        d = (np.exp(m - m_new) * d if d != 0.0 else 0.0) + np.exp(m_chunk - m_new) * d_chunk
+        m = m_new
+    return m, d
+
+
+def tiled_attention_forward(q, k, v, scale: float, causal: bool = False, block: int = 128):
+    """The tiled algorithm with online softmax, written as the pages describe it.
+
+    Loop order of hot.atechcom.net, "How Tiling Works": blocks of K and V outside, blocks of Q
+    inside, with per-row running max m, running sum l and partial output O kept between
+    blocks. Each visit applies the update of iloveeagents.com, "Core Technical Innovations"
+    item 2: m_new = max(m_old, block max); the old l and the old partial O are rescaled by
+    e^{m_old - m_new}; the block's exponentials are taken against m_new. Final O = O / l and
+    lse = m + ln l. Used to pin that the tiled algorithm reaches the definition.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    scale = float(np.float64(scale))
+    n, nk = q.shape[-2], k.shape[-2]
+    o_all = np.zeros(q.shape[:-1] + (v.shape[-1],))
+    lse_all = np.zeros(q.shape[:-1])
+    for idx in _head_iter(q.shape):
+        qh, kh, vh = q[idx], k[idx], v[idx]
+        o = np.zeros((n, vh.shape[1]))
+        m = np.full(n, -np.inf)
+        l = np.zeros(n)
+        for j0 in range(0, nk, block):  # outer: K, V blocks
+            j1 = min(nk, j0 + block)
+            for i0 in range(0, n, block):  # inner: Q blocks
+                i1 = min(n, i0 + block)
+                s = scale * (qh[i0:i1] @ kh[j0:j1].T)
+                if causal:
+                    mask = np.arange(j0, j1)[None, :] <= np.arange(i0, i1)[:, None]
+                    s = np.where(mask, s, -np.inf)
+                else:
+                    mask = np.ones(s.shape, dtype=bool)
+                m_old = m[i0:i1]
+                m_new = np.maximum(m_old, s.max(axis=1))
+                live = np.isfinite(m_new)  # rows with at least one visible key so far
+                m_ref = np.where(live, m_new, 0.0)
+                alpha = np.where(np.isfinite(m_old), np.exp(np.where(np.isfinite(m_old), m_old, 0.0)
+                                                             - m_ref), 0.0)
+                p = np.where(mask, np.exp(np.where(mask, s, 0.0) - m_ref[:, None]), 0.0)
+                l[i0:i1] = alpha * l[i0:i1] + p.sum(axis=1)
+                o[i0:i1] = alpha[:, None] * o[i0:i1] + p @ vh[j0:j1]
+                m[i0:i1] = m_new
+        o_all[idx] = o / l[:, None]
+        lse_all[idx] = m + np.log(l)
+    return o_all, lse_all
