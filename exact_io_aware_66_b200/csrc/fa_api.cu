@@ -1,0 +1,285 @@
+// fa_api.cu — host side of the C ABI declared in include/fa.h: argument validation, TMA
+// tensor-map encoding, kernel launches and error reporting. No device memory is allocated
+// here except one cached 4-byte status word per device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+fa_status set_err(fa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+fa_status cuda_err(cudaError_t e, const char* what) {
+  return set_err(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+struct DeviceState {
+  int* status = nullptr;  // device status word
+  bool checked = false;   // compute capability verified
+  bool is_sm100 = false;
+  bool fwd_attr[2][2] = {{false, false}, {false, false}};  // [d==128][causal]
+  bool bwd_attr[2][2] = {{false, false}, {false, false}};
+};
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Per-device state for the current device; verifies the device is sm_100 and owns the status
+// word. Returns nullptr (with the error set) on failure.
+DeviceState* device_state(fa_status* st) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    *st = cuda_err(e, "cudaGetDevice");
+    return nullptr;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {
+    *st = set_err(FA_ERR_CUDA, "device index %d out of range", dev);
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& ds = g_dev[dev];
+  if (!ds.checked) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    ds.is_sm100 = (major == 10 && minor == 0);
+    ds.checked = true;
+  }
+  if (!ds.is_sm100) {
+    *st = set_err(FA_ERR_CUDA, "device %d is not an sm_100 (B200) GPU", dev);
+    return nullptr;
+  }
+  if (!ds.status) {
+    e = cudaMalloc(&ds.status, sizeof(int));
+    if (e != cudaSuccess) {
+      *st = cuda_err(e, "cudaMalloc(status word)");
+      return nullptr;
+    }
+    e = cudaMemset(ds.status, 0, sizeof(int));
+    if (e != cudaSuccess) {
+      *st = cuda_err(e, "cudaMemset(status word)");
+      return nullptr;
+    }
+  }
+  *st = FA_OK;
+  return &ds;
+}
+
+// 3-D tiled map over a contiguous [BH, N, cols] tensor: dims {cols, N, BH}, box
+// {box_cols, box_rows, 1}. Rows n >= N read as zero and are not written.
+fa_status make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType type, int elem_bytes,
+                   int cols, int N, int BH, int box_cols, int box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return set_err(FA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * elem_bytes,
+                           static_cast<cuuint64_t>(N) * cols * elem_bytes};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, type, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_err(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FA_OK;
+}
+
+fa_status make_bf16_map(CUtensorMap* m, const void* ptr, int d, int N, int BH, int box_rows) {
+  return make_map(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, box_rows,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+fa_status check_sizes(int B, int H, int N, int d, float scale) {
+  if (B < 1 || H < 1 || N < 1)
+    return set_err(FA_ERR_INVALID_ARG, "B, H, N must be >= 1 (got %d, %d, %d)", B, H, N);
+  if (d != 64 && d != 128) return set_err(FA_ERR_UNSUPPORTED, "head dim d=%d not in {64, 128}", d);
+  const long long rows = 1LL * B * H * N;
+  if (rows >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "B*H*N=%lld >= 2^31", rows);
+  if (!std::isfinite(scale) || !(scale > 0.f))
+    return set_err(FA_ERR_INVALID_ARG, "scale must be finite and > 0 (got %g)", (double)scale);
+  return FA_OK;
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
+                     float* lse, int BH, int N, float scale, cudaStream_t stream) {
+  using L = fa::FwdLayout<D>;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
+  bool& attr = ds->fwd_attr[D == 128][CAUSAL];
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncSetAttribute(fwd smem)");
+    attr = true;
+  }
+  CUtensorMap tq, tk, tv, to;
+  fa_status st;
+  if ((st = make_bf16_map(&tq, q, D, N, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tk, k, D, N, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tv, v, D, N, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&to, o, D, N, BH, 32)) != FA_OK) return st;
+  fa::FwdParams p;
+  p.lse = lse;
+  p.status = ds->status;
+  p.N = N;
+  p.BH = BH;
+  p.n_qblocks = (N + 255) / 256;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long grid = 1LL * p.n_qblocks * BH;
+  if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  kern<<<static_cast<unsigned>(grid), fa::kFwdThreads, L::kAlloc, stream>>>(tq, tk, tv, to, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_fwd launch");
+  return FA_OK;
+}
+
+fa_status bwd_dispatch(DeviceState* ds, const void* q, const void* k, const void* v, const void* o,
+                       const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                       void* workspace, int BH, int N, int d, float scale, bool causal,
+                       cudaStream_t stream) {
+  (void)ds; (void)q; (void)k; (void)v; (void)o; (void)dO; (void)lse; (void)dq; (void)dk;
+  (void)dv; (void)workspace; (void)BH; (void)N; (void)d; (void)scale; (void)causal;
+  (void)stream;
+  return set_err(FA_ERR_UNSUPPORTED, "backward kernels not built");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_last_error_string(void) { return g_err; }
+
+const char* fa_version(void) { return "exact_io_aware_66_b200 0.1 (sm_100a)"; }
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float scale, int causal, void* stream) {
+  g_err[0] = '\0';
+  fa_status st = check_sizes(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!q || !k || !v || !o || !lse) return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return set_err(FA_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  const size_t tbytes = static_cast<size_t>(B) * H * N * d * 2;
+  const size_t lbytes = static_cast<size_t>(B) * H * N * 4;
+  const void* ins[3] = {q, k, v};
+  for (const void* in : ins)
+    if (overlaps(o, tbytes, in, tbytes) || overlaps(lse, lbytes, in, tbytes))
+      return set_err(FA_ERR_INVALID_ARG, "outputs must not alias inputs");
+  if (overlaps(o, tbytes, lse, lbytes)) return set_err(FA_ERR_INVALID_ARG, "o and lse overlap");
+  DeviceState* ds = device_state(&st);
+  if (!ds) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (d == 64)
+    return causal ? launch_fwd<64, true>(ds, q, k, v, o, lse, BH, N, scale, s)
+                  : launch_fwd<64, false>(ds, q, k, v, o, lse, BH, N, scale, s);
+  return causal ? launch_fwd<128, true>(ds, q, k, v, o, lse, BH, N, scale, s)
+                : launch_fwd<128, false>(ds, q, k, v, o, lse, BH, N, scale, s);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return fa::bwd_workspace_bytes(rows, d);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+                 void* stream) {
+  g_err[0] = '\0';
+  fa_status st = check_sizes(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv)
+    return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
+  const void* ptrs[10] = {q, k, v, o, dO, lse, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return set_err(FA_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (!workspace || workspace_bytes < need)
+    return set_err(FA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
+                   need);
+  const size_t tbytes = static_cast<size_t>(B) * H * N * d * 2;
+  const size_t lbytes = static_cast<size_t>(B) * H * N * 4;
+  const void* ins[6] = {q, k, v, o, dO, lse};
+  const size_t insz[6] = {tbytes, tbytes, tbytes, tbytes, tbytes, lbytes};
+  void* outs[4] = {dq, dk, dv, workspace};
+  const size_t outsz[4] = {tbytes, tbytes, tbytes, need};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlaps(outs[a], outsz[a], ins[b], insz[b]))
+        return set_err(FA_ERR_INVALID_ARG, "outputs/workspace must not alias inputs");
+    for (int b = a + 1; b < 4; ++b)
+      if (overlaps(outs[a], outsz[a], outs[b], outsz[b]))
+        return set_err(FA_ERR_INVALID_ARG, "outputs/workspace must not overlap each other");
+  }
+  DeviceState* ds = device_state(&st);
+  if (!ds) return st;
+  return bwd_dispatch(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, B * H, N, d, scale,
+                      causal != 0, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_check_status(void* stream) {
+  g_err[0] = '\0';
+  fa_status st;
+  DeviceState* ds = device_state(&st);
+  if (!ds) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_err(e, "cudaStreamSynchronize");
+  int h = 0;
+  e = cudaMemcpy(&h, ds->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_err(e, "read status word");
+  if (h != 0) {
+    e = cudaMemset(ds->status, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_err(e, "clear status word");
+    return set_err(FA_ERR_TIMEOUT, "a bounded in-kernel wait timed out (code %d)", h);
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

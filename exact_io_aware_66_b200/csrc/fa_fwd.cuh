@@ -1,0 +1,435 @@
+// fa_fwd.cuh — exact attention forward for sm_100a (TMA + tcgen05 + TMEM, warp specialised).
+//
+// Computes, for every (batch, head) and query row i,
+//     O_i = sum_j softmax_j(scale * q_i . k_j) v_j      and      lse_i = m_i + ln l_i,
+// tile by tile with the online-softmax running max m and running sum l, so the N x N score
+// and probability matrices never leave the SM ("How FlashAttention Actually Works: Tiling,
+// SRAM Reuse, and Why It's 10x Faster", sections "How Tiling Works" and "The Secret Weapon:
+// Online Softmax"; update rule of "How does FlashAttention optimize memory and speed via
+// tiling?", "Core Technical Innovations" item 2).
+//
+// One CTA owns two 128-row query tiles (256 rows) of one head and streams 128-key K/V tiles
+// through a shared-memory ring. Roles (16 warps):
+//   warps 0-3   softmax for query tile 0   (one thread per row, S read from TMEM)
+//   warps 4-7   softmax for query tile 1
+//   warps 8-11  correction (rescale O in TMEM when the running max grows) and epilogue
+//   warp 12     tcgen05.mma issue (one thread)
+//   warp 13     TMA producer (one thread)
+//   warps 14-15 idle
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// P (bf16) is written back over the first 64 columns of its S buffer and fed to the PV MMA
+// straight from TMEM, so P never touches shared memory.
+// MMA issue order per key tile j: PV0(j), S0(j+1), PV1(j), S1(j+1) — while softmax 0 works on
+// S0(j+1) the tensor core runs PV1(j) and S1(j+1), and vice versa.
+#pragma once
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kFwdThreads = 512;
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTileBytes = 128 * D * 2;  // one 128 x D bf16 tile
+  static constexpr int kBoxBytes = 128 * 64 * 2;  // one TMA box: 128 rows x 64 columns
+  static constexpr int kBoxes = D / 64;           // boxes per tile (128-byte swizzle rows)
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kQ = 0;                                  // Q0, Q1 (reused for O)
+  static constexpr int kKV = 2 * kTileBytes;                    // K/V ring
+  static constexpr int kBars = kKV + kStages * kTileBytes;      // mbarriers
+  static constexpr int kNumBars = 1 + 2 * kStages + 11;
+  static constexpr int kAlpha = kBars + kNumBars * 8;           // float[2][128]
+  static constexpr int kRowL = kAlpha + 2 * 128 * 4;            // float[2][128]
+  static constexpr int kTmemSlot = kRowL + 2 * 128 * 4;
+  static constexpr int kBytes = kTmemSlot + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment of the base
+
+  // barrier indices
+  static constexpr int bQ = 0;
+  static constexpr int bKvFull = 1;                  // + stage
+  static constexpr int bKvEmpty = 1 + kStages;       // + stage
+  static constexpr int bSFull = 1 + 2 * kStages;     // + tile
+  static constexpr int bPFull = bSFull + 2;          // + tile (128 arrivals)
+  static constexpr int bOCorr = bSFull + 4;          // + tile (128 arrivals)
+  static constexpr int bODone = bSFull + 6;          // + tile
+  static constexpr int bFinal = bSFull + 8;          // + tile (128 arrivals)
+  static constexpr int bDrain = bSFull + 10;         // error path only
+};
+
+struct FwdParams {
+  float* lse;       // [BH, N] fp32
+  int* status;      // device status word (FA_ERR_TIMEOUT on a timed-out wait)
+  int N;            // sequence length
+  int BH;           // batch * heads
+  int n_qblocks;    // ceil(N / 256)
+  float scale;      // softmax scale
+  float scale_log2; // scale * log2(e)
+};
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(R));
+}
+
+// Bounded wait whose result is the same on every lane of the warp (needed before the
+// warp-collective tcgen05.ld / tcgen05.st that follow it).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
+__device__ __forceinline__ void fail(int* status, volatile int* abort_flag, int code) {
+  *abort_flag = 1;
+  atomicExch(status, code);
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdParams p) {
+  using L = FwdLayout<D>;
+  constexpr int ST = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int abort_flag_storage;
+  volatile int* abort_flag = &abort_flag_storage;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+  auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * i; };
+  float* s_alpha = reinterpret_cast<float*>(gbase + L::kAlpha);
+  float* s_rowl = reinterpret_cast<float*>(gbase + L::kRowL);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // Heaviest query blocks first (causal work grows with the block index).
+  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x / p.BH);
+  const int bh = static_cast<int>(blockIdx.x % p.BH);
+  const int q0 = qb * 256;
+  const int nkv = (p.N + 127) / 128;
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) n_t[t] = CAUSAL ? min(nkv, 2 * qb + t + 1) : nkv;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(L::bQ), 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(bar(L::bKvFull + s), 1);
+      mbar_init(bar(L::bKvEmpty + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::bSFull + t), 1);
+      mbar_init(bar(L::bPFull + t), 128);
+      mbar_init(bar(L::bOCorr + t), 128);
+      mbar_init(bar(L::bODone + t), 1);
+      mbar_init(bar(L::bFinal + t), 128);
+    }
+    mbar_init(bar(L::bDrain), 1);
+    fence_barrier_init();
+  }
+  if (warp == 12) {
+    tmem_alloc(sbase + L::kTmemSlot, 512);
+    tmem_relinquish();
+  }
+  if (warp == 13 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::kTmemSlot);
+
+  if (warp < 8) {
+    // ------------------------------------------------------------------ softmax ----------
+    setmaxnreg_inc<192>();
+    const int t = warp >> 2;
+    const int row = threadIdx.x & 127;
+    const uint32_t tS = tmem + t * 128 + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const int q_row = q0 + t * 128 + row;
+    const int tile_idx = 2 * qb + t;
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY;
+    float l = 0.f;
+    for (int j = 0; j < n_t[t]; ++j) {
+      if (!warp_wait(bar(L::bSFull + t), j & 1, abort_flag)) {
+        fail(p.status, abort_flag, 5);
+        break;
+      }
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_ld_wait();
+      reg_fence(s);
+      const int kv0 = j * 128;
+      const bool need_mask = (CAUSAL && j == tile_idx) || (kv0 + 128 > p.N);
+      if (need_mask) {
+        const int lim = CAUSAL ? min(q_row + 1, p.N) : p.N;  // keys [0, lim) visible
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
+      }
+      float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
+      float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(s[c]));
+        mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(s[c + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(s[c + 3]));
+      }
+      const float m_new = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
+      const float alpha = ex2_approx((m - m_new) * sl2);  // 0 on the first tile
+      const float nb = -m_new * sl2;
+      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 128; c += 4) {
+        const float e0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, nb));
+        const float e1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, nb));
+        const float e2 = ex2_approx(fmaf(__uint_as_float(s[c + 2]), sl2, nb));
+        const float e3 = ex2_approx(fmaf(__uint_as_float(s[c + 3]), sl2, nb));
+        l0 += e0;
+        l1 += e1;
+        l2 += e2;
+        l3 += e3;
+        pk[c / 2] = pack_bf16x2(e0, e1);
+        pk[c / 2 + 1] = pack_bf16x2(e2, e3);
+      }
+      l = l * alpha + ((l0 + l1) + (l2 + l3));
+      m = m_new;
+      tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+      tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      tmem_st_wait();
+      s_alpha[t * 128 + row] = alpha;
+      tc_fence_before();
+      mbar_arrive(bar(L::bPFull + t));
+    }
+    s_rowl[t * 128 + row] = l;
+    mbar_arrive(bar(L::bFinal + t));
+    if (!*abort_flag && q_row < p.N)
+      p.lse[static_cast<size_t>(bh) * p.N + q_row] = (m * sl2 + lg2_approx(l)) * 0.69314718055994531f;
+  } else if (warp < 12) {
+    // --------------------------------------------------------------- correction ----------
+    setmaxnreg_dec<80>();
+    const int row = threadIdx.x - 256;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    bool ok = true;
+    for (int j = 0; j < n_t[1] && ok; ++j) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (j >= n_t[t]) continue;
+        if (!warp_wait(bar(L::bPFull + t), j & 1, abort_flag)) { ok = false; break; }
+        const float alpha = s_alpha[t * 128 + row];
+        if (j > 0) {
+          if (!warp_wait(bar(L::bODone + t), (j - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+            const uint32_t tO = tmem + 256 + t * D + lane_off;
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              uint32_t o[32];
+              tmem_ld_32x32b_x32(tO + c, o);
+              tmem_ld_wait();
+              reg_fence(o);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st_32x32b_x32(tO + c, o);
+            }
+            tmem_st_wait();
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(L::bOCorr + t));
+      }
+    }
+    if (!ok) fail(p.status, abort_flag, 5);
+    // Epilogue: O = O_acc / l  ->  bf16  ->  swizzled staging (reusing the Q tile)  ->  TMA.
+    // Each warp stores its own 32 rows (box 64 x 32), so no cross-warp barrier is needed.
+    for (int t = 0; t < 2 && ok; ++t) {
+      if (!warp_wait(bar(L::bFinal + t), 0, abort_flag) ||
+          !warp_wait(bar(L::bODone + t), (n_t[t] - 1) & 1, abort_flag)) {
+        fail(p.status, abort_flag, 5);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float inv_l = 1.0f / s_rowl[t * 128 + row];
+      const uint32_t tO = tmem + 256 + t * D + lane_off;
+      uint8_t* stage = gbase + L::kQ + t * L::kTileBytes;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tO + c, o);
+        tmem_ld_wait();
+        reg_fence(o);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // four 16-byte chunks of 8 columns
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+          v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+          v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+          v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+          const int chunk = c / 8 + q;  // 0 .. D/8-1
+          *reinterpret_cast<uint4*>(stage + (chunk >> 3) * L::kBoxBytes +
+                                    sw128_offset(row, chunk & 7)) = v;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int b = 0; b < L::kBoxes; ++b)
+          tma_store_3d(&tmO,
+                       sbase + L::kQ + t * L::kTileBytes + b * L::kBoxBytes + (warp & 3) * 4096,
+                       64 * b, q0 + t * 128 + (warp & 3) * 32, bh);
+        bulk_commit_group();
+      }
+    }
+    if (lane == 0) bulk_wait_group_read0();
+  } else {
+    setmaxnreg_dec<48>();
+    if (warp == 12 && lane == 0) {
+      // ------------------------------------------------------------------ MMA -------------
+      const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+      auto stage_addr = [&](int tt) -> uint32_t {
+        return sbase + L::kKV + static_cast<uint32_t>(tt % ST) * L::kTileBytes;
+      };
+      auto wait_full = [&](int tt) -> bool {
+        return mbar_wait(bar(L::bKvFull + tt % ST), (tt / ST) & 1, abort_flag);
+      };
+      auto issue_s = [&](int t, int j) {
+        const uint32_t qa = sbase + L::kQ + t * L::kTileBytes;
+        const uint32_t ka = stage_addr(2 * j);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
+          umma_ss(tmem + t * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
+                  idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(L::bSFull + t));
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t va = stage_addr(2 * j + 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
+                  sdesc_sw128(va + kk * 2048, L::kBoxBytes, 1024), idesc_pv,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(L::bODone + t));
+      };
+      bool ok = mbar_wait(bar(L::bQ), 0, abort_flag) && wait_full(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit(bar(L::bKvEmpty + 0 % ST));
+      }
+      for (int j = 0; j < n_t[1] && ok; ++j) {
+        const int tv = 2 * j + 1, tk = 2 * j + 2;
+        if (!wait_full(tv)) { ok = false; break; }
+        tc_fence_after();
+        if (j < n_t[0]) {
+          if (!mbar_wait(bar(L::bPFull + 0), j & 1, abort_flag) ||
+              !mbar_wait(bar(L::bOCorr + 0), j & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(0, j);
+        }
+        const bool more = j + 1 < n_t[1];
+        if (more) {
+          if (!wait_full(tk)) { ok = false; break; }
+          tc_fence_after();
+          if (j + 1 < n_t[0]) issue_s(0, j + 1);
+        }
+        if (!mbar_wait(bar(L::bPFull + 1), j & 1, abort_flag) ||
+            !mbar_wait(bar(L::bOCorr + 1), j & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(bar(L::bKvEmpty + tv % ST));
+        if (more) {
+          issue_s(1, j + 1);
+          umma_commit(bar(L::bKvEmpty + tk % ST));
+        }
+      }
+      if (!ok) {
+        fail(p.status, abort_flag, 5);
+        // Drain: wait (bounded) until every MMA issued so far has completed before TMEM and
+        // shared memory are released.
+        volatile int never = 0;
+        umma_commit(bar(L::bDrain));
+        mbar_wait(bar(L::bDrain), 0, &never);
+      }
+    } else if (warp == 13 && lane == 0) {
+      // ------------------------------------------------------------------ TMA -------------
+      mbar_arrive_expect_tx(bar(L::bQ), 2 * L::kTileBytes);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int b = 0; b < L::kBoxes; ++b)
+          tma_load_3d(sbase + L::kQ + t * L::kTileBytes + b * L::kBoxBytes, &tmQ, bar(L::bQ),
+                      64 * b, q0 + 128 * t, bh);
+      int issued = 0;
+      for (int j = 0; j < n_t[1]; ++j) {
+        bool ok = true;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int tt = 2 * j + w;
+          const int st = tt % ST;
+          if (!mbar_wait(bar(L::bKvEmpty + st), ((tt / ST) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(L::bKvFull + st), L::kTileBytes);
+          const uint32_t dst = sbase + L::kKV + st * L::kTileBytes;
+#pragma unroll
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_3d(dst + b * L::kBoxBytes, w ? &tmV : &tmK, bar(L::bKvFull + st), 64 * b,
+                        128 * j, bh);
+          issued = tt + 1;
+        }
+        if (!ok) {
+          fail(p.status, abort_flag, 5);
+          break;
+        }
+      }
+      if (*abort_flag) {
+        // Let the loads already in flight land before shared memory is released.
+        volatile int never = 0;
+        for (int tt = max(0, issued - ST); tt < issued; ++tt)
+          mbar_wait(bar(L::bKvFull + tt % ST), (tt / ST) & 1, &never);
+        mbar_wait(bar(L::bQ), 0, &never);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 12) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

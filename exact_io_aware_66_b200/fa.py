@@ -1,0 +1,165 @@
+"""ctypes binding of libfa.so (include/fa.h). Argument marshalling only: every step of the
+attention forward and backward runs in the library's CUDA kernels.
+
+The functions named like the C entry points (fa_fwd, fa_bwd, fa_bwd_workspace_size,
+fa_check_status, fa_last_error_string) take torch CUDA tensors that the caller allocated;
+``attention_forward`` / ``attention_backward`` allocate the outputs with torch and call them.
+There is no fallback: if libfa.so is missing or the device is not an sm_100 GPU, the calls
+raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa.so")
+
+FA_OK = 0
+STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
+                3: "FA_ERR_MISALIGNED", 4: "FA_ERR_CUDA", 5: "FA_ERR_TIMEOUT",
+                6: "FA_ERR_WORKSPACE"}
+
+# (name, restype, argtypes) of every symbol include/fa.h declares.
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_bwd_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_check_status": (_I, [_P]),
+    "fa_last_error_string": (ctypes.c_char_p, []),
+    "fa_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, where: str, status: int, msg: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libfa.so (built in-tree by exact_io_aware_66_b200.build); raises if absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m exact_io_aware_66_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(where: str, status: int):
+    if status != FA_OK:
+        raise FaError(where, status, fa_last_error_string())
+
+
+def fa_last_error_string() -> str:
+    return (lib().fa_last_error_string() or b"").decode()
+
+
+def fa_version() -> str:
+    return lib().fa_version().decode()
+
+
+def default_scale(d: int) -> float:
+    """1/sqrt(d) rounded to fp32 — the value passed to the kernels."""
+    return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32).item())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dims(x: torch.Tensor):
+    if x.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    return tuple(int(s) for s in x.shape)
+
+
+def _req(x: torch.Tensor, name: str, dtype=torch.bfloat16):
+    if not isinstance(x, torch.Tensor) or not x.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if x.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    if not x.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return x.data_ptr()
+
+
+def fa_fwd(q, k, v, o, lse, causal: bool = False, scale: float | None = None, stream=None):
+    """Forward into caller-allocated o (bf16 [B,H,N,d]) and lse (fp32 [B,H,N])."""
+    B, H, N, d = _dims(q)
+    for t, n in ((k, "k"), (v, "v"), (o, "o")):
+        if _dims(t) != (B, H, N, d):
+            raise ValueError(f"{n} shape mismatch")
+    if tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be [B, H, N]")
+    ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(lse, "lse", torch.float32)]
+    scale = default_scale(d) if scale is None else float(scale)
+    st = lib().fa_fwd(*ptrs, B, H, N, d, scale, int(bool(causal)), _stream_handle(stream))
+    _check("fa_fwd", st)
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_size(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, causal: bool = False,
+           scale: float | None = None, stream=None):
+    """Backward into caller-allocated dq, dk, dv (bf16 [B,H,N,d]) using a caller-owned
+    workspace (uint8 CUDA tensor of at least fa_bwd_workspace_size bytes)."""
+    B, H, N, d = _dims(q)
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (do, "do"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        if _dims(t) != (B, H, N, d):
+            raise ValueError(f"{n} shape mismatch")
+    if tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be [B, H, N]")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(do, "do"),
+            _req(lse, "lse", torch.float32), _req(dq, "dq"), _req(dk, "dk"), _req(dv, "dv")]
+    wbytes = workspace.numel() * workspace.element_size()
+    scale = default_scale(d) if scale is None else float(scale)
+    st = lib().fa_bwd(*ptrs, workspace.data_ptr(), wbytes, B, H, N, d, scale, int(bool(causal)),
+                      _stream_handle(stream))
+    _check("fa_bwd", st)
+
+
+def fa_check_status(stream=None):
+    """Synchronises the stream and raises FaError if an in-kernel wait timed out."""
+    _check("fa_check_status", lib().fa_check_status(_stream_handle(stream)))
+
+
+def attention_forward(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """Returns (o, lse) for bf16 CUDA tensors q, k, v of shape [B, H, N, d]."""
+    B, H, N, d = _dims(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, o, lse, causal, scale, stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
+                       stream=None, workspace=None):
+    """Returns (dq, dk, dv). Allocates the workspace unless one is given."""
+    B, H, N, d = _dims(q)
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8,
+                                device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, causal, scale, stream)
+    return dq, dk, dv

@@ -1,0 +1,88 @@
+/* fa.h — C ABI of the B200 (sm_100a) exact-attention library (libfa.so).
+ *
+ * What is computed (forward): for every batch b, head h and query row i,
+ *     S_ij  = scale * q_i . k_j                    (keys j > i left out when causal)
+ *     O_i   = sum_j softmax_j(S_ij) v_j
+ *     lse_i = m_i + ln l_i,  m_i = max_j S_ij,  l_i = sum_j exp(S_ij - m_i)
+ * i.e. P = softmax(Q K^T / sqrt(d)) and O = P V of "Breaking the Memory Wall: A Deep Dive into
+ * FlashAttention" (section "The Problem: The Memory Wall"), computed tile by tile with the
+ * online-softmax running max m and running sum l of "How FlashAttention Actually Works"
+ * (section "The Secret Weapon: Online Softmax") so that S and P never reach device memory.
+ * The backward recomputes S and P on chip from the stored lse ("The Backward Pass:
+ * Recomputation" on the same page) and returns dQ, dK, dV of the scalar loss whose gradient
+ * with respect to O is dO:
+ *     P = exp(S - lse), dV = P^T dO, dP = dO V^T, D_i = dO_i . O_i, dS = P o (dP - D),
+ *     dQ = scale dS K, dK = scale dS^T Q.
+ *
+ * Layout. q, k, v, o, dO, dq, dk, dv: bf16 [B, H, N, d], contiguous (row-major, d fastest).
+ * lse: fp32 [B, H, N]. Pointers are DEVICE pointers of the current CUDA device, 16-byte aligned.
+ * Causal convention: square, top-left aligned — key j is visible to query i iff j <= i.
+ *
+ * Ownership. The caller owns every buffer, the stream and the backward workspace. The library
+ * keeps, per device, one cached 4-byte status word (allocated on first use) and nothing else.
+ *
+ * Semantics. Calls are asynchronous on `stream` (0 = legacy default stream) and return after
+ * enqueueing. Outputs are fully overwritten. Outputs must not alias inputs. There is no CPU
+ * fallback: without an sm_100 device every compute call returns FA_ERR_CUDA.
+ *
+ * Errors. Arguments are validated before anything is launched; a failed check returns a
+ * non-zero fa_status, launches nothing, and fa_last_error_string() describes it (thread-local).
+ * Every wait inside the kernels is bounded; a wait that times out makes the kernel give up,
+ * record FA_ERR_TIMEOUT in the device status word and return. fa_check_status() synchronises
+ * the stream, reads and clears that word.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null or aliasing pointer, non-positive size, bad scale */
+  FA_ERR_UNSUPPORTED = 2, /* head dim not 64/128, sizes beyond the limits below */
+  FA_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
+  FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (no device, launch error) */
+  FA_ERR_TIMEOUT = 5,     /* a bounded in-kernel wait expired (reported by fa_check_status) */
+  FA_ERR_WORKSPACE = 6    /* backward workspace missing or smaller than fa_bwd_workspace_size */
+} fa_status;
+
+/* Limits: d in {64, 128}; B, H, N >= 1; B*H*N < 2^31; B*H*ceil(N/256) < 2^31. */
+
+/* Forward. Writes o (bf16 [B,H,N,d]) and lse (fp32 [B,H,N]).
+ * scale: the softmax scale (finite, > 0), normally 1/sqrt(d). causal: 0 or 1.
+ * stream: a cudaStream_t passed as void*. */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float scale, int causal, void* stream);
+
+/* Bytes of device workspace fa_bwd needs for these sizes (fp32 dQ accumulator [B,H,N,d] and
+ * the fp32 row term D [B,H,N]). Returns 0 for invalid sizes. */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/* Backward. Inputs q, k, v, o (from fa_fwd), dO and lse (from fa_fwd); outputs dq, dk, dv
+ * (bf16 [B,H,N,d]). workspace: caller-owned device memory of at least
+ * fa_bwd_workspace_size(B,H,N,d) bytes, 16-byte aligned; its contents on entry do not matter. */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+                 void* stream);
+
+/* Synchronises `stream`, then reads and clears the current device's status word.
+ * Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA. */
+fa_status fa_check_status(void* stream);
+
+/* Human-readable description of the last error returned on this thread ("" if none). */
+const char* fa_last_error_string(void);
+
+/* Library version string. */
+const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

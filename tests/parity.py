@@ -1,0 +1,51 @@
+"""Shared helpers for the GPU parity tests: tolerances and error measures.
+
+Tolerances (fixed numbers, never loosened per case):
+  forward O:   max-abs <= 1e-2 and mean-abs <= 1e-3 against the fp64 oracle
+  lse:         max-abs <= 1e-3
+  dQ, dK, dV:  max-abs error / max-abs of the oracle's tensor <= 2e-2, per tensor
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+TOL_O_MAX = 1e-2
+TOL_O_MEAN = 1e-3
+TOL_LSE = 1e-3
+TOL_GRAD_REL = 2e-2
+
+
+def to64(x: torch.Tensor) -> np.ndarray:
+    return x.detach().float().cpu().numpy().astype(np.float64)
+
+
+def fwd_errors(o_gpu, lse_gpu, o_ref, lse_ref) -> dict:
+    o = to64(o_gpu) if isinstance(o_gpu, torch.Tensor) else np.asarray(o_gpu, np.float64)
+    l = to64(lse_gpu) if isinstance(lse_gpu, torch.Tensor) else np.asarray(lse_gpu, np.float64)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(l)), "non-finite output"
+    e = np.abs(o - o_ref)
+    return {"o_max": float(e.max()) if e.size else 0.0,
+            "o_mean": float(e.mean()) if e.size else 0.0,
+            "lse_max": float(np.abs(l - lse_ref).max()) if l.size else 0.0,
+            "o_ref_absmax": float(np.abs(o_ref).max()) if o_ref.size else 0.0}
+
+
+def assert_fwd_ok(err: dict, what: str = ""):
+    assert err["o_max"] <= TOL_O_MAX, f"{what} O max-abs {err['o_max']:.3e}"
+    assert err["o_mean"] <= TOL_O_MEAN, f"{what} O mean-abs {err['o_mean']:.3e}"
+    assert err["lse_max"] <= TOL_LSE, f"{what} lse max-abs {err['lse_max']:.3e}"
+
+
+def grad_rel_error(g_gpu, g_ref) -> float:
+    g = to64(g_gpu) if isinstance(g_gpu, torch.Tensor) else np.asarray(g_gpu, np.float64)
+    assert np.all(np.isfinite(g)), "non-finite gradient"
+    denom = float(np.abs(g_ref).max())
+    return float(np.abs(g - g_ref).max()) / max(denom, 1e-30)
+
+
+def assert_grad_ok(g_gpu, g_ref, what: str):
+    r = grad_rel_error(g_gpu, g_ref)
+    assert r <= TOL_GRAD_REL, f"{what} relative max-norm error {r:.3e}"
+    return r

@@ -1,0 +1,114 @@
+"""The C-ABI library: builds, loads, exports every symbol include/fa.h declares, and rejects
+bad arguments before touching the GPU. CPU only: no compute call reaches a kernel here."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_66_b200 import build as fa_build
+from exact_io_aware_66_b200 import fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return fa.lib()
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "fa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_symbols_exported(lib):
+    names = _header_functions()
+    assert "fa_fwd" in names and "fa_bwd" in names
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in include/fa.h but not exported"
+    assert set(names) <= set(fa.SIGNATURES), "binding lacks a signature for a header function"
+
+
+def test_exports_via_nm():
+    fa_build.build()
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r"\bT (fa_[a-z0-9_]+)", out))
+    assert set(_header_functions()) <= exported
+
+
+def test_version(lib):
+    assert "sm_100a" in fa.fa_version()
+
+
+def test_workspace_size(lib):
+    rows = 2 * 3 * 100
+    ws = fa.fa_bwd_workspace_size(2, 3, 100, 64)
+    assert ws >= rows * 64 * 4 + rows * 4
+    assert ws % 16 == 0
+    assert fa.fa_bwd_workspace_size(2, 3, 100, 96) == 0
+    assert fa.fa_bwd_workspace_size(0, 3, 100, 64) == 0
+
+
+def _fwd_raw(lib, q=16, k=32, v=48, o=1 << 20, lse=2 << 20, B=1, H=1, N=128, d=64, scale=0.125,
+             causal=0):
+    return lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, None)
+
+
+def test_fwd_validation_without_gpu(lib):
+    # every one of these is rejected by the argument checks, before any CUDA call
+    assert _fwd_raw(lib, d=96) == 2
+    assert "head dim" in fa.fa_last_error_string()
+    assert _fwd_raw(lib, N=0) == 1
+    assert _fwd_raw(lib, B=-1) == 1
+    assert _fwd_raw(lib, scale=0.0) == 1
+    assert _fwd_raw(lib, scale=float("nan")) == 1
+    assert _fwd_raw(lib, q=0) == 1
+    assert _fwd_raw(lib, q=8) == 3  # not 16-byte aligned
+    assert _fwd_raw(lib, B=1 << 16, H=1 << 8, N=1 << 8) == 2  # B*H*N >= 2^31
+    # output aliasing an input
+    assert _fwd_raw(lib, o=32) == 1
+
+
+def test_bwd_validation_without_gpu(lib):
+    base = dict(q=1 << 20, k=2 << 20, v=3 << 20, o=4 << 20, do=5 << 20, lse=6 << 20,
+                dq=7 << 20, dk=8 << 20, dv=9 << 20, ws=10 << 20)
+
+    def call(ws_bytes=1 << 20, d=64, N=128, **kw):
+        a = dict(base, **kw)
+        return lib.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"],
+                          a["dv"], a["ws"], ws_bytes, 1, 1, N, d, 0.125, 0, None)
+
+    assert call(d=80) == 2
+    assert call(ws=0) == 6
+    assert call(ws_bytes=16) == 6
+    assert call(dq=0) == 1
+    assert call(dk=(8 << 20) + 4) == 3
+    assert call(dv=1 << 20) == 1  # dv aliases q
+
+
+def test_check_status_without_gpu(lib):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    assert lib.fa_check_status(None) == 4  # FA_ERR_CUDA: no device
+    with pytest.raises(fa.FaError):
+        fa.fa_check_status(0)
+
+
+def test_no_cpu_fallback_in_product_package():
+    """The product package never imports the oracle (no CPU fallback path exists)."""
+    pkg = os.path.join(ROOT, "exact_io_aware_66_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            src = open(os.path.join(pkg, fn)).read()
+            assert not re.search(r"^\s*(from|import)\s+oracle", src, flags=re.M), fn
