@@ -105,13 +105,15 @@ DeviceState* device_state(fa_status* st) {
 // 3-D tiled map over a contiguous [BH, N, cols] tensor: dims {cols, N, BH}, box
 // {box_cols, box_rows, 1}. Rows n >= N read as zero and are not written.
 fa_status make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType type, int elem_bytes,
-                   int cols, int N, int BH, int box_cols, int box_rows, CUtensorMapSwizzle swz) {
+                   int cols, int N, int BH, int box_cols, int box_rows, CUtensorMapSwizzle swz,
+                   long long row_stride = 0) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return set_err(FA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (row_stride == 0) row_stride = cols;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * elem_bytes,
-                           static_cast<cuuint64_t>(N) * cols * elem_bytes};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * elem_bytes,
+                           static_cast<cuuint64_t>(N) * row_stride * elem_bytes};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, type, 3, const_cast<void*>(ptr), dims, strides, box, es,
@@ -178,14 +180,88 @@ fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* 
   return FA_OK;
 }
 
+template <int D, bool CAUSAL>
+fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* v, const void* o,
+                     const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                     void* workspace, int BH, int N, float scale, cudaStream_t stream) {
+  using L = fa::BwdLayout<D>;
+  auto kern = fa::fa_bwd_main<D, CAUSAL>;
+  bool& attr = ds->bwd_attr[D == 128][CAUSAL];
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncSetAttribute(bwd smem)");
+    attr = true;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(ws);
+  float* Dvec = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_D(BH, N, D));
+  float* lse2 = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_lse2(BH, N, D));
+  const int n64 = static_cast<int>(fa::bwd_n64(N));
+  const long long rows = 1LL * BH * N;
+
+  CUtensorMap tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv;
+  fa_status st;
+  if ((st = make_bf16_map(&tq, q, D, N, BH, 64)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tk, k, D, N, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tv, v, D, N, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdo, dO, D, N, BH, 64)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdk, dk, D, N, BH, 32)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdv, dv, D, N, BH, 32)) != FA_OK) return st;
+  // per-row fp32 vectors: [BH][N] with a row stride of N64 elements, 64-element boxes
+  if ((st = make_map(&tl, lse2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 64, 1,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
+    return st;
+  if ((st = make_map(&tD, Dvec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 64, 1,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
+    return st;
+  // dQ accumulator: fp32 [BH][N][D], reduction boxes of 32 columns x 64 rows
+  if ((st = make_map(&tacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, 32, 64,
+                     CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
+    return st;
+
+  constexpr int tpr = D / 8;
+  const long long prep_threads = rows * tpr;
+  const long long prep_blocks = (prep_threads + fa::kPrepThreads - 1) / fa::kPrepThreads;
+  if (prep_blocks >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  fa::fa_bwd_preprocess<D><<<static_cast<unsigned>(prep_blocks), fa::kPrepThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dq_acc,
+      Dvec, lse2, rows, N, n64);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_bwd preprocess launch");
+
+  fa::BwdParams p;
+  p.status = ds->status;
+  p.N = N;
+  p.BH = BH;
+  p.n_kv = (N + 127) / 128;
+  p.n_q = (N + 63) / 64;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long grid = 1LL * p.n_kv * BH;
+  if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  kern<<<static_cast<unsigned>(grid), fa::kBwdThreads, L::kAlloc, stream>>>(
+      tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_bwd main launch");
+
+  const long long n8 = rows * D / 8;
+  fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
+      dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_bwd convert launch");
+  return FA_OK;
+}
+
 fa_status bwd_dispatch(DeviceState* ds, const void* q, const void* k, const void* v, const void* o,
                        const void* dO, const float* lse, void* dq, void* dk, void* dv,
                        void* workspace, int BH, int N, int d, float scale, bool causal,
                        cudaStream_t stream) {
-  (void)ds; (void)q; (void)k; (void)v; (void)o; (void)dO; (void)lse; (void)dq; (void)dk;
-  (void)dv; (void)workspace; (void)BH; (void)N; (void)d; (void)scale; (void)causal;
-  (void)stream;
-  return set_err(FA_ERR_UNSUPPORTED, "backward kernels not built");
+  if (d == 64)
+    return causal ? launch_bwd<64, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream)
+                  : launch_bwd<64, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream);
+  return causal ? launch_bwd<128, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream)
+                : launch_bwd<128, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream);
 }
 
 }  // namespace
@@ -224,8 +300,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
-  const size_t rows = static_cast<size_t>(B) * H * N;
-  return fa::bwd_workspace_bytes(rows, d);
+  return fa::bwd_workspace_bytes(static_cast<size_t>(B) * H, N, d);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,

@@ -1,12 +1,476 @@
 // fa_bwd.cuh — exact attention backward for sm_100a.
+//
+// The backward stores nothing of size N x N: it recomputes the scores and probabilities on chip
+// from Q, K and the forward's per-row logsumexp ("How FlashAttention Actually Works",
+// section "The Backward Pass: Recomputation"; "Breaking the Memory Wall", section "Backward
+// Pass Recomputation": only the normalisation factors are kept). With P = exp(S - lse):
+//     dV = P^T dO,  dP = dO V^T,  D_i = dO_i . O_i,  dS = P o (dP - D),
+//     dQ = scale dS K,  dK = scale dS^T Q
+// (the calculus of softmax attention; the pages give no backward formulas).
+//
+// Three kernels run in order on the caller's stream:
+//   1. fa_bwd_preprocess: D = rowsum(dO o O) (fp32), lse2 = lse * log2(e), dQ_acc = 0.
+//   2. fa_bwd_main: one CTA per (head, 128-key tile j). K_j and V_j stay in shared memory;
+//      64-row tiles of Q and dO stream through a 2-stage TMA ring. Per query tile i, five
+//      tcgen05 MMAs (all M = 128):
+//          S^T  = K_j Q_i^T          -> TMEM (64 columns, double buffered)
+//          dP^T = V_j dO_i^T         -> TMEM (64 columns, double buffered)
+//          dV  += P^T dO_i           (A = P^T from TMEM, bf16)            -> TMEM, d columns
+//          dK  += dS^T Q_i           (A = dS^T from shared memory)       -> TMEM, d columns
+//          dQ^T = K_j^T dS^T         (both operands MN-major in shared memory) -> the dP^T buffer
+//      Two warpgroups turn S^T/dP^T into P^T (back to TMEM) and dS^T (to shared memory) while
+//      the tensor core works on the previous tile; a third drains dQ^T from TMEM and adds it
+//      into the fp32 accumulator with TMA bulk reductions (cp.reduce.async.bulk .add.f32).
+//      The final dK (times scale) and dV are stored with TMA.
+//   3. fa_bwd_dq_convert: dQ = bf16(dQ_acc).
 #pragma once
+#include "fa_fwd.cuh"
 #include "sm100.cuh"
 
 namespace fa {
 
-// Workspace: fp32 dQ accumulator [rows, d] followed by the fp32 row term D [rows].
-inline size_t bwd_workspace_bytes(size_t rows, int d) {
-  return rows * static_cast<size_t>(d) * 4 + ((rows * 4 + 255) / 256) * 256;
+// Workspace layout (all fp32, each section 256-byte aligned):
+//   dQ_acc [BH, N, d] | D [BH, N64] | lse2 [BH, N64]
+// where N64 = N rounded up to a multiple of 64, so every row of D and lse2 starts on a
+// 256-byte boundary (TMA needs 16-byte aligned row strides).
+__host__ __device__ inline size_t bwd_align256(size_t x) { return (x + 255) / 256 * 256; }
+inline size_t bwd_n64(int N) { return (static_cast<size_t>(N) + 63) / 64 * 64; }
+inline size_t bwd_ws_offset_D(size_t BH, int N, int d) {
+  return bwd_align256(BH * N * static_cast<size_t>(d) * 4);
+}
+inline size_t bwd_ws_offset_lse2(size_t BH, int N, int d) {
+  return bwd_ws_offset_D(BH, N, d) + bwd_align256(BH * bwd_n64(N) * 4);
+}
+inline size_t bwd_workspace_bytes(size_t BH, int N, int d) {
+  return bwd_ws_offset_lse2(BH, N, d) + bwd_align256(BH * bwd_n64(N) * 4);
+}
+
+// ------------------------------------------------------------------------------------------
+// 1. Preprocess: one group of d/8 threads per row; each thread owns 8 columns.
+// ------------------------------------------------------------------------------------------
+constexpr int kPrepThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kPrepThreads)
+    fa_bwd_preprocess(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+                      const float* __restrict__ lse, float* __restrict__ dq_acc,
+                      float* __restrict__ Dvec, float* __restrict__ lse2, long long rows, int N,
+                      int n64) {
+  constexpr int TPR = D / 8;  // threads per row
+  const long long t = static_cast<long long>(blockIdx.x) * kPrepThreads + threadIdx.x;
+  const long long row = t / TPR;
+  const int part = static_cast<int>(t % TPR);
+  float acc = 0.f;
+  if (row < rows) {
+    const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
+    const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 fa2 = __bfloat1622float2(a2[i]);
+      const float2 fb2 = __bfloat1622float2(b2[i]);
+      acc = fmaf(fa2.x, fb2.x, acc);
+      acc = fmaf(fa2.y, fb2.y, acc);
+    }
+    float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row < rows && part == 0) {
+    const long long padded = (row / N) * n64 + row % N;
+    Dvec[padded] = acc;
+    lse2[padded] = lse[row] * 1.4426950408889634f;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// 3. dQ conversion: fp32 accumulator (already scaled) -> bf16, 8 elements per thread.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    fa_bwd_dq_convert(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq,
+                      long long n8) {
+  const long long t = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  if (t >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * t];
+  const float4 b = reinterpret_cast<const float4*>(dq_acc)[2 * t + 1];
+  uint4 r;
+  r.x = pack_bf16x2(a.x, a.y);
+  r.y = pack_bf16x2(a.z, a.w);
+  r.z = pack_bf16x2(b.x, b.y);
+  r.w = pack_bf16x2(b.z, b.w);
+  reinterpret_cast<uint4*>(dq)[t] = r;
+}
+
+// ------------------------------------------------------------------------------------------
+// 2. Main kernel.
+// ------------------------------------------------------------------------------------------
+constexpr int kBwdThreads = 512;
+
+template <int D>
+struct BwdLayout {
+  static constexpr int kKVBox = 128 * 64 * 2;   // K/V TMA box: 128 rows x 64 columns
+  static constexpr int kQBox = 64 * 64 * 2;     // Q/dO TMA box: 64 rows x 64 columns
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kKVTile = 128 * D * 2;
+  static constexpr int kQTile = 64 * D * 2;
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kKVTile;
+  static constexpr int kQ = kV + kKVTile;               // + stage * 2 * kQTile
+  static constexpr int kDO = kQ + kQTile;               // + stage * 2 * kQTile
+  static constexpr int kDS = kQ + 4 * kQTile;           // 2 x 16 KB: dS^T [128 keys][64 q]
+  static constexpr int kDQ = kDS + 2 * 16384;           // 4 warps x 8 KB fp32 staging
+  static constexpr int kRow = kDQ + 4 * 8192;           // per stage: lse2[64], D[64]
+  static constexpr int kBars = kRow + 2 * 512;
+  static constexpr int kNumBars = 24;
+  static constexpr int kTmemSlot = kBars + kNumBars * 8;
+  static constexpr int kBytes = kTmemSlot + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+
+  static constexpr int bKV = 0;
+  static constexpr int bQFull = 1;      // + stage
+  static constexpr int bQEmpty = 3;     // + stage
+  static constexpr int bSdPFull = 5;    // + buffer
+  static constexpr int bEwDone = 7;     // + buffer (256 arrivals)
+  static constexpr int bDQFull = 9;     // + buffer
+  static constexpr int bDQFree = 11;    // + buffer (128 arrivals)
+  static constexpr int bDSFree = 13;    // + buffer
+  static constexpr int bAccDone = 15;
+  static constexpr int bDrain = 16;
+
+  // TMEM columns
+  static constexpr uint32_t tDV = 0;
+  static constexpr uint32_t tDK = D;
+  __host__ __device__ static constexpr uint32_t tS(int b) { return 256u + 128u * b; }
+  __host__ __device__ static constexpr uint32_t tDP(int b) { return 256u + 128u * b + 64u; }
+};
+
+struct BwdParams {
+  int* status;
+  int N;
+  int BH;
+  int n_kv;        // ceil(N / 128)
+  int n_q;         // ceil(N / 64)
+  float scale;
+  float scale_log2;
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_main(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                const __grid_constant__ CUtensorMap tmLse2, const __grid_constant__ CUtensorMap tmD,
+                const __grid_constant__ CUtensorMap tmDQacc,
+                const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
+                const BwdParams p) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int abort_flag_storage;
+  volatile int* abort_flag = &abort_flag_storage;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+  auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * i; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int j = static_cast<int>(blockIdx.x / p.BH);  // key tile (heavier first when causal)
+  const int bh = static_cast<int>(blockIdx.x % p.BH);
+  const int k0 = 128 * j;
+  const int qi0 = CAUSAL ? 2 * j : 0;  // first query tile (64 rows) that sees this key tile
+  const int n_i = p.n_q - qi0;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(L::bKV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::bQFull + s), 1);
+      mbar_init(bar(L::bQEmpty + s), 1);
+      mbar_init(bar(L::bSdPFull + s), 1);
+      mbar_init(bar(L::bEwDone + s), 256);
+      mbar_init(bar(L::bDQFull + s), 1);
+      mbar_init(bar(L::bDQFree + s), 128);
+      mbar_init(bar(L::bDSFree + s), 1);
+    }
+    mbar_init(bar(L::bAccDone), 1);
+    mbar_init(bar(L::bDrain), 1);
+    fence_barrier_init();
+  }
+  if (warp == 12) {
+    tmem_alloc(sbase + L::kTmemSlot, 512);
+    tmem_relinquish();
+  }
+  if (warp == 13 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmDQacc);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::kTmemSlot);
+
+  if (warp < 8) {
+    // ------------------------------------------------------- P^T and dS^T (elementwise) ---
+    const int w = warp >> 2;                       // query columns [32w, 32w+32)
+    const int r = threadIdx.x & 127;               // key row within the tile (TMEM lane)
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int key = k0 + r;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int i = 0; i < n_i && ok; ++i) {
+      const int b = i & 1, st = i & 1;
+      const int qi = qi0 + i;
+      ok = warp_wait(bar(L::bQFull + st), (i >> 1) & 1, abort_flag) &&
+           warp_wait(bar(L::bSdPFull + b), (i >> 1) & 1, abort_flag) &&
+           (i < 2 || warp_wait(bar(L::bDSFree + b), ((i >> 1) & 1) ^ 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[32], dp[32];
+      tmem_ld_32x32b_x32(tmem + L::tS(b) + 32 * w + lane_off, s);
+      tmem_ld_32x32b_x32(tmem + L::tDP(b) + 32 * w + lane_off, dp);
+      tmem_ld_wait();
+      reg_fence(s);
+      reg_fence(dp);
+      const float* lse2 = reinterpret_cast<const float*>(gbase + L::kRow + st * 512) + 32 * w;
+      const float* Dv = reinterpret_cast<const float*>(gbase + L::kRow + st * 512 + 256) + 32 * w;
+      const int qbase = 64 * qi + 32 * w;
+      const bool need_mask = (CAUSAL && qi <= 2 * j + 1) || (qbase + 32 > p.N) || (k0 + 128 > p.N);
+      uint32_t pk[16], dsk[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        float pr[2], dsr[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int cc = c + e;
+          const int q = qbase + cc;
+          const bool masked = need_mask && (q >= p.N || key >= p.N || (CAUSAL && q < key));
+          const float pv = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(s[cc]), sl2, -lse2[cc]));
+          pr[e] = pv;
+          dsr[e] = masked ? 0.f : pv * (__uint_as_float(dp[cc]) - Dv[cc]);
+        }
+        pk[c / 2] = pack_bf16x2(pr[0], pr[1]);
+        dsk[c / 2] = pack_bf16x2(dsr[0], dsr[1]);
+      }
+      tmem_st_32x32b_x16(tmem + L::tS(b) + 32 * w + lane_off, pk);
+      uint8_t* dsb = gbase + L::kDS + b * 16384;
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        *reinterpret_cast<uint4*>(dsb + sw128_offset(r, 4 * w + t)) =
+            make_uint4(dsk[4 * t], dsk[4 * t + 1], dsk[4 * t + 2], dsk[4 * t + 3]);
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(L::bEwDone + b));
+    }
+    if (!ok) fail(p.status, abort_flag, 5);
+    // ------------------------------------------------------------ dV / dK epilogue -------
+    if (ok && warp_wait(bar(L::bAccDone), 0, abort_flag)) {
+      tc_fence_after();
+      // warpgroup 0 stores dV (stage-0 Q/dO space), warpgroup 1 stores dK * scale (stage 1)
+      const uint32_t tcol = w == 0 ? L::tDV : L::tDK;
+      const float mul = w == 0 ? 1.0f : p.scale;
+      const int region = L::kQ + w * 2 * L::kQTile;
+      uint8_t* stage = gbase + region;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + tcol + c + lane_off, v);
+        tmem_ld_wait();
+        reg_fence(v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 u;
+          u.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * mul, __uint_as_float(v[8 * q + 1]) * mul);
+          u.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * mul, __uint_as_float(v[8 * q + 3]) * mul);
+          u.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * mul, __uint_as_float(v[8 * q + 5]) * mul);
+          u.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * mul, __uint_as_float(v[8 * q + 7]) * mul);
+          const int chunk = c / 8 + q;
+          *reinterpret_cast<uint4*>(stage + (chunk >> 3) * L::kKVBox + sw128_offset(r, chunk & 7)) = u;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const CUtensorMap* map = w == 0 ? &tmDV : &tmDK;
+#pragma unroll
+        for (int bx = 0; bx < L::kBoxes; ++bx)
+          tma_store_3d(map, sbase + region + bx * L::kKVBox + (warp & 3) * 4096, 64 * bx,
+                       k0 + (warp & 3) * 32, bh);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+      }
+    } else if (ok) {
+      fail(p.status, abort_flag, 5);
+    }
+  } else if (warp < 12) {
+    // ---------------------------------------------------------------- dQ drain ----------
+    const int wq = warp & 3;                         // d columns [32 wq, 32 wq + 32)
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    float* stagef = reinterpret_cast<float*>(gbase + L::kDQ + wq * 8192);
+    const uint32_t stage_s = sbase + L::kDQ + wq * 8192;
+    const bool active = 32 * wq < D;
+    bool ok = true;
+    for (int i = 0; i < n_i; ++i) {
+      const int b = i & 1;
+      if (!warp_wait(bar(L::bDQFull + b), (i >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld_32x32b_x32(tmem + L::tDP(b) + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld_32x32b_x32(tmem + L::tDP(b) + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_ld_wait();
+      reg_fence(v);
+      tc_fence_before();
+      mbar_arrive(bar(L::bDQFree + b));
+      if (!active) continue;
+      if (lane == 0) bulk_wait_group_read0();  // previous reduction finished reading staging
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 64; ++q) stagef[q * 32 + lane] = __uint_as_float(v[q]) * p.scale;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_3d(&tmDQacc, stage_s, 32 * wq, 64 * (qi0 + i), bh);
+        bulk_commit_group();
+      }
+    }
+    if (!ok) fail(p.status, abort_flag, 5);
+    if (lane == 0) bulk_wait_group0();
+  } else if (warp == 12) {
+    // --------------------------------------------------------------------- MMA ----------
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32(128, 64, false, false);   // S^T, dP^T
+      const uint32_t id_acc = idesc_bf16_f32(128, D, false, true);   // dV, dK
+      const uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);    // dQ^T
+      auto first_half = [&](int i) {
+        const int b = i & 1, st = i & 1;
+        const uint32_t qa = sbase + L::kQ + st * 2 * L::kQTile;
+        const uint32_t da = sbase + L::kDO + st * 2 * L::kQTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t okv = (kk >> 2) * L::kKVBox + (kk & 3) * 32;
+          const uint32_t oq = (kk >> 2) * L::kQBox + (kk & 3) * 32;
+          umma_ss(tmem + L::tS(b), sdesc_sw128(sbase + L::kK + okv, 16, 1024),
+                  sdesc_sw128(qa + oq, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t okv = (kk >> 2) * L::kKVBox + (kk & 3) * 32;
+          const uint32_t oq = (kk >> 2) * L::kQBox + (kk & 3) * 32;
+          umma_ss(tmem + L::tDP(b), sdesc_sw128(sbase + L::kV + okv, 16, 1024),
+                  sdesc_sw128(da + oq, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(L::bSdPFull + b));
+      };
+      auto second_half = [&](int i) {
+        const int b = i & 1, st = i & 1;
+        const uint32_t qa = sbase + L::kQ + st * 2 * L::kQTile;
+        const uint32_t da = sbase + L::kDO + st * 2 * L::kQTile;
+        const uint32_t dsa = sbase + L::kDS + b * 16384;
+        // dV += P^T dO: P^T (keys x 64 queries) from TMEM; query columns 0-31 were packed into
+        // S columns [0,16), 32-63 into [32,48).
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ts(tmem + L::tDV, tmem + L::tS(b) + (kk >> 1) * 32 + (kk & 1) * 8,
+                  sdesc_sw128(da + kk * 2048, L::kQBox, 1024), id_acc,
+                  (i > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ss(tmem + L::tDK, sdesc_sw128(dsa + kk * 32, 16, 1024),
+                  sdesc_sw128(qa + kk * 2048, L::kQBox, 1024), id_acc,
+                  (i > 0 || kk > 0) ? 1u : 0u);
+        // dQ^T = K^T dS^T  (M = 128 rows of d; for d = 64 the second half of the rows repeats
+        // the first and is ignored by the drain)
+        const uint32_t lbo_k = D == 128 ? static_cast<uint32_t>(L::kKVBox) : 0u;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tmem + L::tDP(b), sdesc_sw128(sbase + L::kK + kk * 2048, lbo_k, 1024),
+                  sdesc_sw128(dsa + kk * 2048, 16, 1024), id_dq, kk > 0 ? 1u : 0u);
+        umma_commit(bar(L::bDQFull + b));
+        umma_commit(bar(L::bQEmpty + st));
+        umma_commit(bar(L::bDSFree + b));
+      };
+      bool ok = mbar_wait(bar(L::bKV), 0, abort_flag);
+      for (int i = 0; i < n_i && ok; ++i) {
+        const int b = i & 1, st = i & 1;
+        ok = mbar_wait(bar(L::bQFull + st), (i >> 1) & 1, abort_flag) &&
+             (i < 2 || mbar_wait(bar(L::bDQFree + b), ((i >> 1) & 1) ^ 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        first_half(i);
+        if (i > 0) {
+          const int pb = (i - 1) & 1;
+          if (!mbar_wait(bar(L::bEwDone + pb), ((i - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          second_half(i - 1);
+        }
+      }
+      if (ok) {
+        const int i = n_i - 1;
+        ok = mbar_wait(bar(L::bEwDone + (i & 1)), (i >> 1) & 1, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          second_half(i);
+          umma_commit(bar(L::bAccDone));
+        }
+      }
+      if (!ok) {
+        fail(p.status, abort_flag, 5);
+        volatile int never = 0;
+        umma_commit(bar(L::bDrain));
+        mbar_wait(bar(L::bDrain), 0, &never);
+      }
+    }
+  } else if (warp == 13) {
+    // --------------------------------------------------------------------- TMA ----------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(L::bKV), 2 * L::kKVTile);
+#pragma unroll
+      for (int bx = 0; bx < L::kBoxes; ++bx) {
+        tma_load_3d(sbase + L::kK + bx * L::kKVBox, &tmK, bar(L::bKV), 64 * bx, k0, bh);
+        tma_load_3d(sbase + L::kV + bx * L::kKVBox, &tmV, bar(L::bKV), 64 * bx, k0, bh);
+      }
+      int issued = 0;
+      for (int i = 0; i < n_i; ++i) {
+        const int st = i & 1;
+        if (!mbar_wait(bar(L::bQEmpty + st), ((i >> 1) & 1) ^ 1, abort_flag)) {
+          fail(p.status, abort_flag, 5);
+          break;
+        }
+        const int q0 = 64 * (qi0 + i);
+        mbar_arrive_expect_tx(bar(L::bQFull + st), 2 * L::kQTile + 512);
+#pragma unroll
+        for (int bx = 0; bx < L::kBoxes; ++bx) {
+          tma_load_3d(sbase + L::kQ + st * 2 * L::kQTile + bx * L::kQBox, &tmQ,
+                      bar(L::bQFull + st), 64 * bx, q0, bh);
+          tma_load_3d(sbase + L::kDO + st * 2 * L::kQTile + bx * L::kQBox, &tmDO,
+                      bar(L::bQFull + st), 64 * bx, q0, bh);
+        }
+        tma_load_3d(sbase + L::kRow + st * 512, &tmLse2, bar(L::bQFull + st), q0, bh, 0);
+        tma_load_3d(sbase + L::kRow + st * 512 + 256, &tmD, bar(L::bQFull + st), q0, bh, 0);
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        for (int i = max(0, issued - 2); i < issued; ++i)
+          mbar_wait(bar(L::bQFull + (i & 1)), (i >> 1) & 1, &never);
+        mbar_wait(bar(L::bKV), 0, &never);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 12) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 }  // namespace fa

@@ -1,0 +1,144 @@
+"""Backward parity: dQ, dK, dV from the CUDA path (through the C ABI) against the fp64 oracle.
+Tolerance: max-abs error / max-abs of the oracle's tensor <= 2e-2, per tensor."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_66_b200 import fa
+from exact_io_aware_66_b200.workloads import (WORKLOADS, make_inputs, sampled_keys, sampled_rows,
+                                              workload_inputs)
+from parity import TOL_GRAD_REL, assert_grad_ok, grad_rel_error, to64
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [  # (B, H, N, d): several tiles, ragged tails, N = 1
+    (1, 1, 1, 64), (1, 2, 5, 128), (2, 1, 64, 64), (1, 2, 128, 128), (1, 1, 200, 64),
+    (2, 2, 300, 128), (1, 1, 640, 64), (1, 2, 1000, 128), (1, 1, 1152, 128),
+]
+
+
+def _fwd_bwd(x, causal, scale=None):
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_forward(q, k, v, causal=causal, scale=scale)
+    dq, dk, dv = fa.attention_backward(q, k, v, o, do, lse, causal=causal, scale=scale)
+    fa.fa_check_status()
+    return o, lse, dq, dk, dv
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "b%dh%dn%dd%d" % s)
+def test_bwd_small_full_compare(shape, causal):
+    B, H, N, d = shape
+    x = make_inputs(B, H, N, d, seed=200 + N + d)
+    _, _, dq, dk, dv = _fwd_bwd(x, causal)
+    ref = oracle.attention_backward(to64(x["q"]), to64(x["k"]), to64(x["v"]), to64(x["do"]),
+                                    fa.default_scale(d), causal)
+    for g, r, n in zip((dq, dk, dv), ref, ("dQ", "dK", "dV")):
+        assert_grad_ok(g, r, f"{shape} causal={causal} {n}")
+
+
+def _head_subset(w, n_heads, seed):
+    rng = np.random.Generator(np.random.PCG64(w.seed + seed))
+    return [divmod(int(t), w.H) for t in rng.choice(w.B * w.H, size=n_heads, replace=False)]
+
+
+@pytest.mark.parametrize("name", ["train_b8h16n2048d64", "causal_train_b4h16n4096d128"])
+def test_bwd_full_size_whole_heads(name):
+    """Full-size training workloads in the bench's launch configuration: dQ, dK, dV of whole
+    seeded heads against the oracle, and dQ of sampled rows across every head."""
+    w = WORKLOADS[name]
+    x = workload_inputs(w)
+    _, _, dq, dk, dv = _fwd_bwd(x, w.causal)
+    for g in (dq, dk, dv):
+        assert torch.isfinite(g).all()
+    dq64, dk64, dv64 = to64(dq), to64(dk), to64(dv)
+    for b, h in _head_subset(w, 2, 3000):
+        ref = oracle.attention_backward(to64(x["q"][b, h]), to64(x["k"][b, h]), to64(x["v"][b, h]),
+                                        to64(x["do"][b, h]), w.scale, w.causal)
+        for g, r, n in zip((dq64[b, h], dk64[b, h], dv64[b, h]), ref, ("dQ", "dK", "dV")):
+            assert_grad_ok(g, r, f"{name} head ({b},{h}) {n}")
+    rows = sampled_rows(w, 256)
+    q, k, v, do = (x[n].float().numpy() for n in ("q", "k", "v", "do"))
+    _, _, dq_ref = oracle.attention_rows(q, k, v, w.scale, w.causal, rows, do=do)
+    idx = tuple(np.array(rows).T)
+    assert grad_rel_error(dq64[idx], dq_ref) <= TOL_GRAD_REL
+
+
+def test_bwd_long_sequence_sampled():
+    """B=1, H=16, N=16384, d=128 causal: dQ on 512 sampled rows, dK and dV on 64 sampled keys
+    (drawn from 2 seeded heads, whose full forward the oracle needs)."""
+    w = WORKLOADS["causal_train_b1h16n16384d128"]
+    x = workload_inputs(w)
+    _, _, dq, dk, dv = _fwd_bwd(x, w.causal)
+    q, k, v, do = (x[n].float().numpy() for n in ("q", "k", "v", "do"))
+    rows = sampled_rows(w, w.row_samples)
+    _, _, dq_ref = oracle.attention_rows(q, k, v, w.scale, w.causal, rows, do=do)
+    idx = tuple(np.array(rows).T)
+    assert grad_rel_error(to64(dq)[idx], dq_ref) <= TOL_GRAD_REL
+    keys = sampled_keys(w, w.key_samples, max_heads=2)
+    dk64, dv64 = to64(dk), to64(dv)
+    for head in sorted({(b, h) for b, h, _ in keys}):
+        js = [jj for b, h, jj in keys if (b, h) == head]
+        dk_ref, dv_ref = oracle.attention_keys(q, k, v, do, w.scale, w.causal, head, js)
+        assert grad_rel_error(dk64[head][js], dk_ref) <= TOL_GRAD_REL, f"dK head {head}"
+        assert grad_rel_error(dv64[head][js], dv_ref) <= TOL_GRAD_REL, f"dV head {head}"
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_causal_masked_queries_have_no_effect(d):
+    """Under the causal mask, queries i < j0 never see keys >= j0: changing Q and dO rows
+    i < j0 leaves dK and dV rows >= j0 bit-identical."""
+    B, H, N, j0 = 1, 2, 640, 333
+    x = make_inputs(B, H, N, d, seed=12)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_forward(q, k, v, causal=True)
+    _, dk1, dv1 = fa.attention_backward(q, k, v, o, do, lse, causal=True)
+    g = torch.Generator().manual_seed(5)
+    q2, do2 = q.clone(), do.clone()
+    q2[:, :, :j0] = (torch.randn(q2[:, :, :j0].shape, generator=g) * 2).to(q.dtype).cuda()
+    do2[:, :, :j0] = (torch.randn(do2[:, :, :j0].shape, generator=g) * 2).to(q.dtype).cuda()
+    _, dk2, dv2 = fa.attention_backward(q2, k, v, o, do2, lse, causal=True)
+    fa.fa_check_status()
+    assert torch.equal(dk1[:, :, j0:], dk2[:, :, j0:])
+    assert torch.equal(dv1[:, :, j0:], dv2[:, :, j0:])
+    assert not torch.equal(dk1[:, :, :j0], dk2[:, :, :j0])
+
+
+def test_bwd_dk_dv_deterministic():
+    x = make_inputs(1, 4, 1024, 128, seed=13)
+    _, _, dq1, dk1, dv1 = _fwd_bwd(x, True)
+    _, _, dq2, dk2, dv2 = _fwd_bwd(x, True)
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    # dQ is accumulated by unordered reductions: equal within tolerance, not bit for bit
+    assert grad_rel_error(dq1, to64(dq2)) <= 1e-3
+
+
+def test_bwd_workspace_reuse_and_dirty_workspace():
+    """The workspace's contents on entry do not matter."""
+    x = make_inputs(1, 2, 384, 64, seed=14)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_forward(q, k, v)
+    ws = torch.full((fa.fa_bwd_workspace_size(1, 2, 384, 64),), 255, dtype=torch.uint8,
+                    device="cuda")
+    dq1, dk1, dv1 = fa.attention_backward(q, k, v, o, do, lse, workspace=ws)
+    dq2, dk2, dv2 = fa.attention_backward(q, k, v, o, do, lse, workspace=ws)
+    fa.fa_check_status()
+    ref = oracle.attention_backward(to64(x["q"]), to64(x["k"]), to64(x["v"]), to64(x["do"]),
+                                    fa.default_scale(64), False)
+    for g, r in zip((dq1, dk1, dv1), ref):
+        assert grad_rel_error(g, r) <= TOL_GRAD_REL
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+
+
+def test_bwd_rejects_small_workspace():
+    x = make_inputs(1, 1, 128, 64, seed=15)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_forward(q, k, v)
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fa.FaError) as e:
+        fa.attention_backward(q, k, v, o, do, lse, workspace=ws)
+    assert e.value.status == 6
