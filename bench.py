@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the attention hot path: one step = forward (fa_fwd) + backward (fa_bwd) of
+exact attention on one batch of seeded synthetic bf16 inputs, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints ONE JSON line (rank 0). ``value`` is whole-job attention TFLOP/s (fwd + bwd) with
+inputs resident in device memory; ``e2e`` is the same metric with pinned-host inputs copied in
+and every output copied back inside the timed region. Multi-GPU runs (torchrun) are
+independent replicas of the same workload, one per GPU (weak scaling); the only collectives
+are the barrier and the max-over-ranks of the timing.
+
+FLOP accounting: forward 4 B H N^2 d, backward 2.5x forward, both halved when causal.
+``--impl reference`` times the fp64 CPU oracle on the host instead, on bounded samples of the
+same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from exact_io_aware_66_b200.workloads import WORKLOADS, workload_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "causal_train_b4h16n4096d128"
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 512 * 1024 * 1024
+KERNEL_SOURCES = ["exact_io_aware_66_b200/csrc/fa_bwd.cuh", "exact_io_aware_66_b200/csrc/fa_fwd.cuh",
+                  "exact_io_aware_66_b200/csrc/sm100.cuh", "exact_io_aware_66_b200/csrc/fa_api.cu"]
+
+
+def load_metric() -> str:
+    try:
+        with open(os.path.join(ROOT, "BASELINE.json")) as f:
+            return json.load(f)["metric"]
+    except Exception:
+        return "attention TFLOP/s (fwd, fwd+bwd) bf16"
+
+
+def load_peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"bf16_burst": float(d["bf16_tflops"]),
+                "bf16_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"bf16_burst": 1590.0, "bf16_sustained": 1400.0, "hbm_gbs": 6650.0,
+                "source": "fallback"}
+
+
+def sources_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
+    current kernel sources (same source hash); else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel][workload]
+        if e.get("sources_hash") != sources_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------------------------------------
+# Clock sampling (nvidia-smi) during the timed region
+# --------------------------------------------------------------------------------------------
+REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.gpu = str(device)
+
+    def start(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.out = open(os.devnull, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        mhz, maxmhz, reasons = [], [], set()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                maxmhz.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(REASONS, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxmhz),
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# --------------------------------------------------------------------------------------------
+# Distributed plumbing (replicas only)
+# --------------------------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle, as it stands
+# --------------------------------------------------------------------------------------------
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_head_step(x, w, heads, prefix: int | None = None):
+    """Oracle fwd+bwd of the given (b, h) heads, optionally restricted to the first `prefix`
+    rows and keys (a self-contained sub-problem under the causal mask). Returns FLOPs done."""
+    import numpy as np
+
+    import oracle
+
+    n = w.N if prefix is None else prefix
+    for b, h in heads:
+        q, k, v = (x[t][b, h, :n].float().numpy().astype(np.float64) for t in ("q", "k", "v"))
+        if w.backward:
+            do = x["do"][b, h, :n].float().numpy().astype(np.float64)
+            oracle.attention_backward(q, k, v, do, w.scale, w.causal)
+        else:
+            oracle.attention_forward(q, k, v, w.scale, w.causal)
+    f = 4.0 * n * n * w.d * (3.5 if w.backward else 1.0) * len(heads)
+    return f / 2 if w.causal else f
+
+
+def cpu_baseline(w, x, budget_s: float = 12.0) -> dict:
+    heads_all = [(b, h) for b in range(w.B) for h in range(w.H)]
+    t0 = time.perf_counter()
+    flops = oracle_head_step(x, w, heads_all[:1], prefix=min(w.N, 4096))
+    one = time.perf_counter() - t0
+    prefix = min(w.N, 4096)
+    nh = max(1, min(len(heads_all), int(budget_s / max(one, 1e-3))))
+    heads = heads_all[:nh]
+    t0 = time.perf_counter()
+    flops = oracle_head_step(x, w, heads, prefix=prefix)
+    dt = time.perf_counter() - t0
+    sample = (f"oracle fwd{'+bwd' if w.backward else ''} (fp64 NumPy) of {nh} of {len(heads_all)} "
+              f"heads" + (f", first {prefix} rows/keys of each" if prefix < w.N else "")
+              + f"; {dt:.1f} s")
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(),
+            "kind": "oracle", "sample": sample}
+
+
+def run_reference(args, w, world, rank):
+    """The reference arm: the fp64 CPU oracle on bounded samples of the same workload."""
+    if rank != 0:
+        return 0
+    x = workload_inputs(w)
+    steps, warm = args.steps, args.warmup
+    budget_per_step = max(0.05, 150.0 / (steps + warm))
+    # calibrate a causal-prefix length (multiple of 128) so one step takes about the budget
+    t0 = time.perf_counter()
+    oracle_head_step(x, w, [(0, 0)], prefix=min(w.N, 1024))
+    t1024 = time.perf_counter() - t0
+    n = int(min(w.N, 1024 * (budget_per_step / max(t1024, 1e-4)) ** 0.5))
+    n = max(128, n // 128 * 128)
+    heads = [(0, 0)]
+    for _ in range(warm):
+        oracle_head_step(x, w, heads, prefix=n)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for s in range(steps):
+        b, h = divmod(s % (w.B * w.H), w.H)
+        flops += oracle_head_step(x, w, [(b, h)], prefix=n)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = (f"per step: oracle fwd{'+bwd' if w.backward else ''} (fp64 NumPy) of one head, "
+              f"first {n} of {w.N} rows/keys")
+    line = {"impl": "reference", "metric": load_metric(), "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": dt * 1000 / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1), bf16-rounded, widened to fp64)",
+            "config": workload_config(w, world),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, world) -> dict:
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "pass": "fwd+bwd" if w.backward else "fwd", "scale": "1/sqrt(d)",
+            "flops_per_step": w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"{FLUSH_BYTES >> 20} MiB buffer written before every timed step "
+                  f"(L2 is {L2_BYTES >> 20} MiB)"}
+
+
+# --------------------------------------------------------------------------------------------
+# Our arm
+# --------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, w, world, rank)
+
+    from exact_io_aware_66_b200 import fa
+
+    fa.lib()  # fails loudly if the CUDA library is missing: there is no fallback
+    dev = torch.device("cuda", local)
+    x = workload_inputs(w)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    do = x["do"].to(dev) if w.backward else None
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    if w.backward:
+        ws = torch.empty(fa.fa_bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8,
+                         device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(q_, k_, v_, do_):
+        fa.fa_fwd(q_, k_, v_, o, lse, w.causal, None, stream)
+        if w.backward:
+            fa.fa_bwd(q_, k_, v_, o, do_, lse, dq, dk, dv, ws, w.causal, None, stream)
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step(q, k, v, do)
+    fa.fa_check_status(stream)
+    flops_step = workload_config(w, world)["flops_per_step"]
+    launches_per_step = 1 + (3 if w.backward else 0)
+
+    # ---- timed region: K steps, L2 flushed before each (outside the event pairs) ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    fa.fa_profile_read()
+    fa.fa_profile_enable(True)
+    for s in range(args.steps):
+        flush.zero_()
+        starts[s].record(stream)
+        step(q, k, v, do)
+        ends[s].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop()
+    fa.fa_profile_enable(False)
+    prof = fa.fa_profile_read()
+    fa.fa_check_status(stream)
+    ms_total = sum(a.elapsed_time(b) for a, b in zip(starts, ends))
+    ms_total = max_over_ranks(ms_total, world)
+    value = flops_step * args.steps * world / (ms_total / 1e3) / 1e12
+    ms_step = ms_total / args.steps
+
+    # per-kernel device time from the library's own event pairs
+    kern = {name: {"launches": n, "ms": t} for name, (n, t) in prof.items() if n}
+    fwd_ms = kern.get("fa_fwd_kernel", {}).get("ms", 0.0) / args.steps
+    bwd_ms = sum(kern.get(n, {}).get("ms", 0.0)
+                 for n in ("fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert")) / args.steps
+    peaks = load_peaks()
+    dom = max(kern, key=lambda n: kern[n]["ms"])
+    dom_flops = {"fa_fwd_kernel": w.fwd_flops(), "fa_bwd_main": w.bwd_flops()}.get(dom)
+    avg_ms = kern[dom]["ms"] / kern[dom]["launches"]
+    peak = peaks["bf16_sustained"] if ms_total > 1000 else peaks["bf16_burst"]
+    achieved = dom_flops / (avg_ms / 1e3) / 1e12 if dom_flops else None
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak if achieved else None,
+                "traffic": ncu_traffic(dom, w.name),
+                "peak_source": f"{peaks['source']} bf16 "
+                               f"{'sustained' if ms_total > 1000 else 'burst'} (MEASURED_PEAKS.json)",
+                "per_launch_flops": dom_flops, "avg_launch_ms": avg_ms}
+
+    # ---- end-to-end: pinned host inputs in, every output back, inside the timed region ----
+    host_in = {n: x[n].pin_memory() for n in (("q", "k", "v", "do") if w.backward else ("q", "k", "v"))}
+    outs = [o, lse] + ([dq, dk, dv] if w.backward else [])
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+
+    def e2e_step():
+        for n, t in host_in.items():
+            dev_in[n].copy_(t, non_blocking=True)
+        step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in.get("do"))
+        for t, h in zip(outs, host_out):
+            h.copy_(t, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    fa.fa_check_status(stream)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e = {"value": flops_step * args.e2e_steps * world / (e2e_ms / 1e3) / 1e12,
+           "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, x)
+
+    if rank == 0:
+        line = {
+            "metric": load_metric(), "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1)" + (f" x{w.mult}" if w.mult != 1 else "")
+                    + ", bf16), inputs resident in device memory",
+            "config": workload_config(w, world),
+            "fwd_tflops": w.fwd_flops() / (fwd_ms / 1e3) / 1e12 if fwd_ms else None,
+            "bwd_tflops": (w.bwd_flops() / (bwd_ms / 1e3) / 1e12) if bwd_ms else None,
+            "frac_of_peak": {"fwd+bwd": value / world / peaks["bf16_burst"],
+                             "fwd": (w.fwd_flops() / (fwd_ms / 1e3) / 1e12) / peaks["bf16_burst"]
+                             if fwd_ms else None,
+                             "peak": peaks["bf16_burst"], "peak_source":
+                                 f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"},
+            "roofline": roofline,
+            "kernels": kern,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/fa.h"
 #include "fa_bwd.cuh"
@@ -29,6 +30,51 @@ fa_status set_err(fa_status s, const char* fmt, ...) {
 fa_status cuda_err(cudaError_t e, const char* what) {
   return set_err(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
+
+// ---- optional per-kernel device timing (fa_profile_enable / fa_profile_read) ----
+constexpr int kKernelKinds = 4;  // fwd, bwd preprocess, bwd main, bwd dQ convert
+const char* const kKernelNames[kKernelKinds] = {"fa_fwd_kernel", "fa_bwd_preprocess",
+                                                "fa_bwd_main", "fa_bwd_dq_convert"};
+struct ProfileRec {
+  int kind;
+  cudaEvent_t start, stop;
+};
+struct ProfileState {
+  bool on = false;
+  std::vector<ProfileRec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+};
+thread_local ProfileState g_prof;
+
+// RAII bracket around one kernel launch: records an event pair on `stream` when profiling is on.
+struct ProfileScope {
+  int kind;
+  cudaStream_t stream;
+  cudaEvent_t start = nullptr;
+  ProfileScope(int k, cudaStream_t s) : kind(k), stream(s) {
+    if (g_prof.on && (start = g_prof.get())) cudaEventRecord(start, stream);
+  }
+  ~ProfileScope() {
+    if (!start) return;
+    cudaEvent_t stop = g_prof.get();
+    if (!stop) {
+      g_prof.pool.push_back(start);
+      return;
+    }
+    cudaEventRecord(stop, stream);
+    g_prof.recs.push_back({kind, start, stop});
+  }
+};
 
 constexpr int kMaxDevices = 64;
 struct DeviceState {
@@ -174,6 +220,7 @@ fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* 
   p.scale_log2 = scale * 1.4426950408889634f;
   const long long grid = 1LL * p.n_qblocks * BH;
   if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  ProfileScope prof(0, stream);
   kern<<<static_cast<unsigned>(grid), fa::kFwdThreads, L::kAlloc, stream>>>(tq, tk, tv, to, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_fwd launch");
@@ -224,9 +271,12 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   const long long prep_threads = rows * tpr;
   const long long prep_blocks = (prep_threads + fa::kPrepThreads - 1) / fa::kPrepThreads;
   if (prep_blocks >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
-  fa::fa_bwd_preprocess<D><<<static_cast<unsigned>(prep_blocks), fa::kPrepThreads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dq_acc,
-      Dvec, lse2, rows, N, n64);
+  {
+    ProfileScope prof(1, stream);
+    fa::fa_bwd_preprocess<D><<<static_cast<unsigned>(prep_blocks), fa::kPrepThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dq_acc,
+        Dvec, lse2, rows, N, n64);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd preprocess launch");
 
@@ -236,18 +286,31 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   p.BH = BH;
   p.n_kv = (N + 127) / 128;
   p.n_q = (N + 63) / 64;
+  {
+    // heads per scheduling group: Q, dO, K, V (bf16) and the fp32 dQ accumulator of a group
+    // should stay within about half of the 126 MB L2
+    const double per_head = static_cast<double>(N) * D * (2 + 2 + 2 + 2 + 4);
+    const int g = static_cast<int>(64.0 * 1024 * 1024 / per_head);
+    p.group = g < 1 ? 1 : (g > BH ? BH : g);
+  }
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   const long long grid = 1LL * p.n_kv * BH;
   if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
-  kern<<<static_cast<unsigned>(grid), fa::kBwdThreads, L::kAlloc, stream>>>(
-      tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv, p);
+  {
+    ProfileScope prof(2, stream);
+    kern<<<static_cast<unsigned>(grid), fa::kBwdThreads, L::kAlloc, stream>>>(
+        tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv, p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd main launch");
 
   const long long n8 = rows * D / 8;
-  fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
-      dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+  {
+    ProfileScope prof(3, stream);
+    fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
+        dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd convert launch");
   return FA_OK;
@@ -337,6 +400,38 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (!ds) return st;
   return bwd_dispatch(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, B * H, N, d, scale,
                       causal != 0, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_profile_enable(int on) {
+  g_prof.on = on != 0;
+  return FA_OK;
+}
+
+fa_status fa_profile_read(double* ms, long long* launches, int n) {
+  g_err[0] = '\0';
+  if (!ms || !launches || n < kKernelKinds)
+    return set_err(FA_ERR_INVALID_ARG, "fa_profile_read needs arrays of %d entries", kKernelKinds);
+  for (int i = 0; i < n; ++i) {
+    ms[i] = 0.0;
+    launches[i] = 0;
+  }
+  fa_status st = FA_OK;
+  for (const ProfileRec& r : g_prof.recs) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.stop);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.start, r.stop);
+    if (e != cudaSuccess && st == FA_OK) st = cuda_err(e, "profile event");
+    ms[r.kind] += t;
+    launches[r.kind] += 1;
+    g_prof.pool.push_back(r.start);
+    g_prof.pool.push_back(r.stop);
+  }
+  g_prof.recs.clear();
+  return st;
+}
+
+const char* fa_kernel_name(int kind) {
+  return (kind >= 0 && kind < kKernelKinds) ? kKernelNames[kind] : "";
 }
 
 fa_status fa_check_status(void* stream) {

@@ -9,7 +9,7 @@
 // (the calculus of softmax attention; the pages give no backward formulas).
 //
 // Three kernels run in order on the caller's stream:
-//   1. fa_bwd_preprocess: D = rowsum(dO o O) (fp32), lse2 = lse * log2(e), dQ_acc = 0.
+//   1. fa_bwd_preprocess: D = rowsum(dO o O) (fp32), lse2 = -lse * log2(e), dQ_acc = 0.
 //   2. fa_bwd_main: one CTA per (head, 128-key tile j). K_j and V_j stay in shared memory;
 //      64-row tiles of Q and dO stream through a 2-stage TMA ring. Per query tile i, five
 //      tcgen05 MMAs (all M = 128):
@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kPrepThreads)
   if (row < rows && part == 0) {
     const long long padded = (row / N) * n64 + row % N;
     Dvec[padded] = acc;
-    lse2[padded] = lse[row] * 1.4426950408889634f;
+    lse2[padded] = -lse[row] * 1.4426950408889634f;  // stored negated: P = 2^(S log2e scale + this)
   }
 }
 
@@ -116,29 +116,31 @@ struct BwdLayout {
   static constexpr int kBoxes = D / 64;
   static constexpr int kKVTile = 128 * D * 2;
   static constexpr int kQTile = 64 * D * 2;
+  static constexpr int kQStages = (D == 128) ? 3 : 4;  // Q/dO ring depth
   static constexpr int kK = 0;
   static constexpr int kV = kK + kKVTile;
   static constexpr int kQ = kV + kKVTile;               // + stage * 2 * kQTile
   static constexpr int kDO = kQ + kQTile;               // + stage * 2 * kQTile
-  static constexpr int kDS = kQ + 4 * kQTile;           // 2 x 16 KB: dS^T [128 keys][64 q]
+  static constexpr int kDS = kQ + kQStages * 2 * kQTile;  // 2 x 16 KB: dS^T [128 keys][64 q]
   static constexpr int kDQ = kDS + 2 * 16384;           // 4 warps x 8 KB fp32 staging
   static constexpr int kRow = kDQ + 4 * 8192;           // per stage: lse2[64], D[64]
-  static constexpr int kBars = kRow + 2 * 512;
-  static constexpr int kNumBars = 24;
+  static constexpr int kBars = kRow + kQStages * 512;
+
+  static constexpr int bKV = 0;
+  static constexpr int bQFull = 1;                      // + stage
+  static constexpr int bQEmpty = 1 + kQStages;          // + stage
+  static constexpr int bSdPFull = 1 + 2 * kQStages;     // + buffer
+  static constexpr int bEwDone = bSdPFull + 2;          // + buffer (256 arrivals)
+  static constexpr int bDQFull = bSdPFull + 4;          // + buffer
+  static constexpr int bDQFree = bSdPFull + 6;          // + buffer (128 arrivals)
+  static constexpr int bDSFree = bSdPFull + 8;          // + buffer
+  static constexpr int bAccDone = bSdPFull + 10;
+  static constexpr int bDrain = bSdPFull + 11;
+  static constexpr int kNumBars = bDrain + 1;
+
   static constexpr int kTmemSlot = kBars + kNumBars * 8;
   static constexpr int kBytes = kTmemSlot + 16;
   static constexpr int kAlloc = kBytes + 1024;
-
-  static constexpr int bKV = 0;
-  static constexpr int bQFull = 1;      // + stage
-  static constexpr int bQEmpty = 3;     // + stage
-  static constexpr int bSdPFull = 5;    // + buffer
-  static constexpr int bEwDone = 7;     // + buffer (256 arrivals)
-  static constexpr int bDQFull = 9;     // + buffer
-  static constexpr int bDQFree = 11;    // + buffer (128 arrivals)
-  static constexpr int bDSFree = 13;    // + buffer
-  static constexpr int bAccDone = 15;
-  static constexpr int bDrain = 16;
 
   // TMEM columns
   static constexpr uint32_t tDV = 0;
@@ -153,6 +155,7 @@ struct BwdParams {
   int BH;
   int n_kv;        // ceil(N / 128)
   int n_q;         // ceil(N / 64)
+  int group;       // heads per scheduling group
   float scale;
   float scale_log2;
 };
@@ -177,8 +180,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int j = static_cast<int>(blockIdx.x / p.BH);  // key tile (heavier first when causal)
-  const int bh = static_cast<int>(blockIdx.x % p.BH);
+  // Heads are processed in groups of p.group, sized on the host so that a group's Q, dO, K, V
+  // and dQ accumulator fit in L2; within a group the key tiles with the most query tiles
+  // (causal) come first, cycling over the group's heads (longest-processing-time order).
+  constexpr int QS = L::kQStages;
+  const int per_group = p.group * p.n_kv;
+  const int g0 = static_cast<int>(blockIdx.x / per_group) * p.group;
+  const int r_in = static_cast<int>(blockIdx.x % per_group);
+  const int gcur = min(p.group, p.BH - g0);
+  const int j = r_in / gcur;
+  const int bh = g0 + r_in % gcur;
   const int k0 = 128 * j;
   const int qi0 = CAUSAL ? 2 * j : 0;  // first query tile (64 rows) that sees this key tile
   const int n_i = p.n_q - qi0;
@@ -186,9 +197,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(bar(L::bKV), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < QS; ++s) {
       mbar_init(bar(L::bQFull + s), 1);
       mbar_init(bar(L::bQEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(bar(L::bSdPFull + s), 1);
       mbar_init(bar(L::bEwDone + s), 256);
       mbar_init(bar(L::bDQFull + s), 1);
@@ -224,9 +237,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int i = 0; i < n_i && ok; ++i) {
-      const int b = i & 1, st = i & 1;
+      const int b = i & 1, st = i % QS;
       const int qi = qi0 + i;
-      ok = warp_wait(bar(L::bQFull + st), (i >> 1) & 1, abort_flag) &&
+      ok = warp_wait(bar(L::bQFull + st), (i / QS) & 1, abort_flag) &&
            warp_wait(bar(L::bSdPFull + b), (i >> 1) & 1, abort_flag) &&
            (i < 2 || warp_wait(bar(L::bDSFree + b), ((i >> 1) & 1) ^ 1, abort_flag));
       if (!ok) break;
@@ -242,20 +255,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int qbase = 64 * qi + 32 * w;
       const bool need_mask = (CAUSAL && qi <= 2 * j + 1) || (qbase + 32 > p.N) || (k0 + 128 > p.N);
       uint32_t pk[16], dsk[16];
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float pr[2], dsr[2];
+      for (int c = 0; c < 32; c += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);  // -lse * log2(e)
+        const float4 d4 = *reinterpret_cast<const float4*>(Dv + c);
+        float a[4], pr[4], dsr[4];
+        f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, f2_pack(l4.x, l4.y)), a[0], a[1]);
+        f2_unpack(f2_fma(f2_pack_u(s[c + 2], s[c + 3]), sl2x2, f2_pack(l4.z, l4.w)), a[2], a[3]);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int cc = c + e;
-          const int q = qbase + cc;
-          const bool masked = need_mask && (q >= p.N || key >= p.N || (CAUSAL && q < key));
-          const float pv = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(s[cc]), sl2, -lse2[cc]));
-          pr[e] = pv;
-          dsr[e] = masked ? 0.f : pv * (__uint_as_float(dp[cc]) - Dv[cc]);
+        for (int e = 0; e < 4; ++e) pr[e] = ex2_approx(a[e]);
+        f2_unpack(f2_mul(f2_pack(pr[0], pr[1]),
+                         f2_sub(f2_pack_u(dp[c], dp[c + 1]), f2_pack(d4.x, d4.y))),
+                  dsr[0], dsr[1]);
+        f2_unpack(f2_mul(f2_pack(pr[2], pr[3]),
+                         f2_sub(f2_pack_u(dp[c + 2], dp[c + 3]), f2_pack(d4.z, d4.w))),
+                  dsr[2], dsr[3]);
+        if (need_mask) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int q = qbase + c + e;
+            if (q >= p.N || key >= p.N || (CAUSAL && q < key)) {
+              pr[e] = 0.f;
+              dsr[e] = 0.f;
+            }
+          }
         }
         pk[c / 2] = pack_bf16x2(pr[0], pr[1]);
+        pk[c / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
         dsk[c / 2] = pack_bf16x2(dsr[0], dsr[1]);
+        dsk[c / 2 + 1] = pack_bf16x2(dsr[2], dsr[3]);
       }
       tmem_st_32x32b_x16(tmem + L::tS(b) + 32 * w + lane_off, pk);
       uint8_t* dsb = gbase + L::kDS + b * 16384;
@@ -348,7 +377,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t id_acc = idesc_bf16_f32(128, D, false, true);   // dV, dK
       const uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);    // dQ^T
       auto first_half = [&](int i) {
-        const int b = i & 1, st = i & 1;
+        const int b = i & 1, st = i % QS;
         const uint32_t qa = sbase + L::kQ + st * 2 * L::kQTile;
         const uint32_t da = sbase + L::kDO + st * 2 * L::kQTile;
 #pragma unroll
@@ -368,7 +397,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         umma_commit(bar(L::bSdPFull + b));
       };
       auto second_half = [&](int i) {
-        const int b = i & 1, st = i & 1;
+        const int b = i & 1, st = i % QS;
         const uint32_t qa = sbase + L::kQ + st * 2 * L::kQTile;
         const uint32_t da = sbase + L::kDO + st * 2 * L::kQTile;
         const uint32_t dsa = sbase + L::kDS + b * 16384;
@@ -398,8 +427,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       };
       bool ok = mbar_wait(bar(L::bKV), 0, abort_flag);
       for (int i = 0; i < n_i && ok; ++i) {
-        const int b = i & 1, st = i & 1;
-        ok = mbar_wait(bar(L::bQFull + st), (i >> 1) & 1, abort_flag) &&
+        const int b = i & 1, st = i % QS;
+        ok = mbar_wait(bar(L::bQFull + st), (i / QS) & 1, abort_flag) &&
              (i < 2 || mbar_wait(bar(L::bDQFree + b), ((i >> 1) & 1) ^ 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
@@ -438,8 +467,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       int issued = 0;
       for (int i = 0; i < n_i; ++i) {
-        const int st = i & 1;
-        if (!mbar_wait(bar(L::bQEmpty + st), ((i >> 1) & 1) ^ 1, abort_flag)) {
+        const int st = i % QS;
+        if (!mbar_wait(bar(L::bQEmpty + st), ((i / QS) & 1) ^ 1, abort_flag)) {
           fail(p.status, abort_flag, 5);
           break;
         }
@@ -458,8 +487,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (*abort_flag) {
         volatile int never = 0;
-        for (int i = max(0, issued - 2); i < issued; ++i)
-          mbar_wait(bar(L::bQFull + (i & 1)), (i >> 1) & 1, &never);
+        for (int i = max(0, issued - QS); i < issued; ++i)
+          mbar_wait(bar(L::bQFull + (i % QS)), (i / QS) & 1, &never);
         mbar_wait(bar(L::bKV), 0, &never);
       }
     }

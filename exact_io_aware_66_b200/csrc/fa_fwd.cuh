@@ -12,7 +12,7 @@
 // through a shared-memory ring. Roles (16 warps):
 //   warps 0-3   softmax for query tile 0   (one thread per row, S read from TMEM)
 //   warps 4-7   softmax for query tile 1
-//   warps 8-11  correction (rescale O in TMEM when the running max grows) and epilogue
+//   warps 8-11  epilogue (O / l -> bf16 -> TMA store)
 //   warp 12     tcgen05.mma issue (one thread)
 //   warp 13     TMA producer (one thread)
 //   warps 14-15 idle
@@ -27,6 +27,8 @@
 namespace fa {
 
 constexpr int kFwdThreads = 512;
+// Running-max update threshold, log2 units (exponentials stay below 2^8 between updates).
+constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
 struct FwdLayout {
@@ -38,8 +40,7 @@ struct FwdLayout {
   static constexpr int kKV = 2 * kTileBytes;                    // K/V ring
   static constexpr int kBars = kKV + kStages * kTileBytes;      // mbarriers
   static constexpr int kNumBars = 1 + 2 * kStages + 11;
-  static constexpr int kAlpha = kBars + kNumBars * 8;           // float[2][128]
-  static constexpr int kRowL = kAlpha + 2 * 128 * 4;            // float[2][128]
+  static constexpr int kRowL = kBars + kNumBars * 8;            // float[2][128]
   static constexpr int kTmemSlot = kRowL + 2 * 128 * 4;
   static constexpr int kBytes = kTmemSlot + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment of the base
@@ -50,7 +51,6 @@ struct FwdLayout {
   static constexpr int bKvEmpty = 1 + kStages;       // + stage
   static constexpr int bSFull = 1 + 2 * kStages;     // + tile
   static constexpr int bPFull = bSFull + 2;          // + tile (128 arrivals)
-  static constexpr int bOCorr = bSFull + 4;          // + tile (128 arrivals)
   static constexpr int bODone = bSFull + 6;          // + tile
   static constexpr int bFinal = bSFull + 8;          // + tile (128 arrivals)
   static constexpr int bDrain = bSFull + 10;         // error path only
@@ -112,12 +112,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (sbase - raw);
   auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * i; };
-  float* s_alpha = reinterpret_cast<float*>(gbase + L::kAlpha);
   float* s_rowl = reinterpret_cast<float*>(gbase + L::kRowL);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Heaviest query blocks first (causal work grows with the block index).
+  // Longest-processing-time order: all heads' heaviest query blocks (causal work grows with
+  // the block index) are scheduled first.
   const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x / p.BH);
   const int bh = static_cast<int>(blockIdx.x % p.BH);
   const int q0 = qb * 256;
@@ -136,7 +136,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::bSFull + t), 1);
       mbar_init(bar(L::bPFull + t), 128);
-      mbar_init(bar(L::bOCorr + t), 128);
       mbar_init(bar(L::bODone + t), 1);
       mbar_init(bar(L::bFinal + t), 128);
     }
@@ -160,7 +159,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (warp < 8) {
     // ------------------------------------------------------------------ softmax ----------
-    setmaxnreg_inc<192>();
+    setmaxnreg_inc<176>();
     const int t = warp >> 2;
     const int row = threadIdx.x & 127;
     const uint32_t tS = tmem + t * 128 + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -168,7 +167,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int tile_idx = 2 * qb + t;
     const float sl2 = p.scale_log2;
     float m = -INFINITY;
-    float l = 0.f;
+    float l = 0.f;   // sum of the fp32 exponentials: gives lse
+    float lr = 0.f;  // sum of the same exponentials rounded to bf16: normalises O, whose
+                     // PV MMA used exactly those rounded weights
     for (int j = 0; j < n_t[t]; ++j) {
       if (!warp_wait(bar(L::bSFull + t), j & 1, abort_flag)) {
         fail(p.status, abort_flag, 5);
@@ -193,78 +194,81 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
       float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(s[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(s[c + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(s[c + 3]));
+      for (int c = 4; c < 128; c += 8) {
+        mx0 = max3f(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        mx1 = max3f(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        mx2 = max3f(mx2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+        mx3 = max3f(mx3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
       }
-      const float m_new = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
-      const float alpha = ex2_approx((m - m_new) * sl2);  // 0 on the first tile
-      const float nb = -m_new * sl2;
-      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+      // The running max is raised only when a tile's max exceeds it by more than
+      // kRescaleLog2 (in log2 units): until then exponentials stay below 2^kRescaleLog2, and
+      // the final O / l and lse = m + ln l use the same (stale) m, so the result is exact.
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      float alpha = 1.0f;
+      if ((m_tile - m) * sl2 > kRescaleLog2) {  // always true on the first tile (m = -inf)
+        alpha = ex2_approx((m - m_tile) * sl2);  // 0 on the first tile
+        m = m_tile;
+      }
+      const float nb = -m * sl2;
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), nbx2 = f2_pack(nb, nb);
+      uint64_t lsum[4] = {0, 0, 0, 0}, rsum[4] = {0, 0, 0, 0};  // (0.f, 0.f) pairs
       uint32_t pk[64];
 #pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        const float e0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, nb));
-        const float e1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, nb));
-        const float e2 = ex2_approx(fmaf(__uint_as_float(s[c + 2]), sl2, nb));
-        const float e3 = ex2_approx(fmaf(__uint_as_float(s[c + 3]), sl2, nb));
-        l0 += e0;
-        l1 += e1;
-        l2 += e2;
-        l3 += e3;
-        pk[c / 2] = pack_bf16x2(e0, e1);
-        pk[c / 2 + 1] = pack_bf16x2(e2, e3);
+      for (int c = 0; c < 128; c += 2) {
+        float a0, a1;
+        f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, nbx2), a0, a1);
+        const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
+        const uint32_t w = pack_bf16x2(e0, e1);
+        pk[c / 2] = w;
+        lsum[(c >> 1) & 3] = f2_add(lsum[(c >> 1) & 3], f2_pack(e0, e1));
+        rsum[(c >> 1) & 3] = f2_add(rsum[(c >> 1) & 3], f2_pack_u(w << 16, w & 0xffff0000u));
       }
-      l = l * alpha + ((l0 + l1) + (l2 + l3));
-      m = m_new;
+      {
+        const uint64_t ls = f2_add(f2_add(lsum[0], lsum[1]), f2_add(lsum[2], lsum[3]));
+        const uint64_t rs = f2_add(f2_add(rsum[0], rsum[1]), f2_add(rsum[2], rsum[3]));
+        float x0, x1, y0, y1;
+        f2_unpack(ls, x0, x1);
+        f2_unpack(rs, y0, y1);
+        l = l * alpha + (x0 + x1);
+        lr = lr * alpha + (y0 + y1);
+      }
       tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
       tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      // O correction. S(j) was issued after PV(j-1) and tcgen05 MMAs complete in order, so
+      // PV(j-1) has finished: O can be rescaled here without another wait. PV(j) is issued
+      // only after the arrive below.
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        const uint32_t tO = tmem + 256 + t * D + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(tO + c, o);
+          tmem_ld_wait();
+          reg_fence(o);
+          const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const uint64_t r = f2_mul(f2_pack_u(o[i], o[i + 1]), a2);
+            o[i] = static_cast<uint32_t>(r);
+            o[i + 1] = static_cast<uint32_t>(r >> 32);
+          }
+          tmem_st_32x32b_x32(tO + c, o);
+        }
+      }
       tmem_st_wait();
-      s_alpha[t * 128 + row] = alpha;
       tc_fence_before();
       mbar_arrive(bar(L::bPFull + t));
     }
-    s_rowl[t * 128 + row] = l;
+    s_rowl[t * 128 + row] = lr;
     mbar_arrive(bar(L::bFinal + t));
     if (!*abort_flag && q_row < p.N)
       p.lse[static_cast<size_t>(bh) * p.N + q_row] = (m * sl2 + lg2_approx(l)) * 0.69314718055994531f;
   } else if (warp < 12) {
-    // --------------------------------------------------------------- correction ----------
+    // ----------------------------------------------------------------- epilogue ----------
     setmaxnreg_dec<80>();
     const int row = threadIdx.x - 256;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
-    for (int j = 0; j < n_t[1] && ok; ++j) {
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (j >= n_t[t]) continue;
-        if (!warp_wait(bar(L::bPFull + t), j & 1, abort_flag)) { ok = false; break; }
-        const float alpha = s_alpha[t * 128 + row];
-        if (j > 0) {
-          if (!warp_wait(bar(L::bODone + t), (j - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-            const uint32_t tO = tmem + 256 + t * D + lane_off;
-#pragma unroll
-            for (int c = 0; c < D; c += 32) {
-              uint32_t o[32];
-              tmem_ld_32x32b_x32(tO + c, o);
-              tmem_ld_wait();
-              reg_fence(o);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st_32x32b_x32(tO + c, o);
-            }
-            tmem_st_wait();
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(bar(L::bOCorr + t));
-      }
-    }
-    if (!ok) fail(p.status, abort_flag, 5);
     // Epilogue: O = O_acc / l  ->  bf16  ->  swizzled staging (reusing the Q tile)  ->  TMA.
     // Each warp stores its own 32 rows (box 64 x 32), so no cross-warp barrier is needed.
     for (int t = 0; t < 2 && ok; ++t) {
@@ -309,7 +313,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     if (lane == 0) bulk_wait_group_read0();
   } else {
-    setmaxnreg_dec<48>();
+    setmaxnreg_dec<80>();
     if (warp == 12 && lane == 0) {
       // ------------------------------------------------------------------ MMA -------------
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
@@ -352,8 +356,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!wait_full(tv)) { ok = false; break; }
         tc_fence_after();
         if (j < n_t[0]) {
-          if (!mbar_wait(bar(L::bPFull + 0), j & 1, abort_flag) ||
-              !mbar_wait(bar(L::bOCorr + 0), j & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar(L::bPFull + 0), j & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           issue_pv(0, j);
         }
@@ -363,8 +366,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tc_fence_after();
           if (j + 1 < n_t[0]) issue_s(0, j + 1);
         }
-        if (!mbar_wait(bar(L::bPFull + 1), j & 1, abort_flag) ||
-            !mbar_wait(bar(L::bOCorr + 1), j & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(L::bPFull + 1), j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         issue_pv(1, j);
         umma_commit(bar(L::bKvEmpty + tv % ST));

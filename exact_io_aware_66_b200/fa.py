@@ -33,7 +33,12 @@ SIGNATURES = {
     "fa_check_status": (_I, [_P]),
     "fa_last_error_string": (ctypes.c_char_p, []),
     "fa_version": (ctypes.c_char_p, []),
+    "fa_profile_enable": (_I, [_I]),
+    "fa_profile_read": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), _I]),
+    "fa_kernel_name": (ctypes.c_char_p, [_I]),
 }
+
+KERNEL_KINDS = 4
 
 _lib = None
 
@@ -137,6 +142,19 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, causal: bool = False,
     st = lib().fa_bwd(*ptrs, workspace.data_ptr(), wbytes, B, H, N, d, scale, int(bool(causal)),
                       _stream_handle(stream))
     _check("fa_bwd", st)
+
+
+def fa_profile_enable(on: bool = True):
+    _check("fa_profile_enable", lib().fa_profile_enable(int(bool(on))))
+
+
+def fa_profile_read() -> dict:
+    """{kernel name: (launches, summed device ms)} since the last read."""
+    ms = (ctypes.c_double * KERNEL_KINDS)()
+    n = (ctypes.c_longlong * KERNEL_KINDS)()
+    _check("fa_profile_read", lib().fa_profile_read(ms, n, KERNEL_KINDS))
+    return {lib().fa_kernel_name(i).decode(): (int(n[i]), float(ms[i]))
+            for i in range(KERNEL_KINDS)}
 
 
 def fa_check_status(stream=None):

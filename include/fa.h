@@ -75,6 +75,20 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA. */
 fa_status fa_check_status(void* stream);
 
+/* Optional device-side timing of the library's own kernels, for benchmarks and tracing.
+ * While enabled on the calling thread, every kernel fa_fwd / fa_bwd launches is bracketed by a
+ * pair of CUDA events recorded on its launch stream. fa_profile_read() waits for those events
+ * and writes, per kernel kind k (0 = forward, 1 = backward preprocess, 2 = backward main,
+ * 3 = backward dQ conversion; FA_KERNEL_KINDS in total), the number of launches to
+ * launches[k] and their summed device time in milliseconds to ms[k], then forgets them.
+ * n is the length of both arrays (>= FA_KERNEL_KINDS). Events are created by the library and
+ * reused; no device memory is allocated. */
+#define FA_KERNEL_KINDS 4
+fa_status fa_profile_enable(int on);
+fa_status fa_profile_read(double* ms, long long* launches, int n);
+/* Name of kernel kind k ("" if out of range). */
+const char* fa_kernel_name(int kind);
+
 /* Human-readable description of the last error returned on this thread ("" if none). */
 const char* fa_last_error_string(void);
 
