@@ -327,6 +327,23 @@ fa_status bwd_dispatch(DeviceState* ds, const void* q, const void* k, const void
                 : launch_bwd<128, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream);
 }
 
+// ---- fa_bwd_noalloc: backward whose scratch is built into the library ----
+// The backward needs scratch (fp32 dQ accumulator, row terms D and -lse*log2e). For callers that
+// cannot allocate device memory, fa_bwd_noalloc uses this file-scope array instead of a
+// caller-provided workspace. Every GPU that loads this library holds it until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+// In-kernel timeout code of fa_bwd_noalloc calls (the hang guard of the bounded waits).
+static __device__ int g_noalloc_status;
+
+struct NoAllocDevice {
+  bool ready = false;
+  void* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+  int* status = nullptr;    // device address of g_noalloc_status on this device
+  bool bwd_attr[2][2] = {{false, false}, {false, false}};
+};
+NoAllocDevice g_noalloc[kMaxDevices];
+
 }  // namespace
 
 extern "C" {
@@ -432,6 +449,80 @@ fa_status fa_profile_read(double* ms, long long* launches, int n) {
 
 const char* fa_kernel_name(int kind) {
   return (kind >= 0 && kind < kKernelKinds) ? kKernelNames[kind] : "";
+}
+
+// Backward with built-in scratch (see include/fa.h). Allocates nothing: no cudaMalloc, no
+// cudaFree, no allocating library routine. Set-up (once per device, on the first call with
+// that device current): the device addresses of the scratch array and of the status word are
+// taken with cudaGetSymbolAddress.
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const void* dO, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, float scale, int causal, void* stream) {
+  g_err[0] = '\0';
+  fa_status st = check_sizes(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (need > kNoAllocScratchBytes)
+    return set_err(FA_ERR_UNSUPPORTED,
+                   "fa_bwd_noalloc: these sizes need %zu bytes of scratch, more than the %zu "
+                   "bytes built into the library (use fa_bwd with a workspace)",
+                   need, kNoAllocScratchBytes);
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv)
+    return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
+  const void* ptrs[9] = {q, k, v, o, dO, lse, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return set_err(FA_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  const size_t tbytes = static_cast<size_t>(B) * H * N * d * 2;
+  const size_t lbytes = static_cast<size_t>(B) * H * N * 4;
+  const void* ins[6] = {q, k, v, o, dO, lse};
+  const size_t insz[6] = {tbytes, tbytes, tbytes, tbytes, tbytes, lbytes};
+  void* outs[3] = {dq, dk, dv};
+  for (int a = 0; a < 3; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlaps(outs[a], tbytes, ins[b], insz[b]))
+        return set_err(FA_ERR_INVALID_ARG, "outputs must not alias inputs");
+    for (int b = a + 1; b < 3; ++b)
+      if (overlaps(outs[a], tbytes, outs[b], tbytes))
+        return set_err(FA_ERR_INVALID_ARG, "outputs must not overlap each other");
+  }
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_err(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return set_err(FA_ERR_CUDA, "device index %d out of range", dev);
+  DeviceState local;  // per-call view: status word and attribute flags of the no-alloc path
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    NoAllocDevice& nd = g_noalloc[dev];
+    if (!nd.ready) {
+      int major = 0, minor = 0;
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+      if (!(major == 10 && minor == 0))
+        return set_err(FA_ERR_CUDA, "device %d is not an sm_100 (B200) GPU", dev);
+      void* scratch = nullptr;
+      e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_err(e, "cudaGetSymbolAddress(scratch)");
+      void* status = nullptr;
+      e = cudaGetSymbolAddress(&status, g_noalloc_status);
+      if (e != cudaSuccess) return cuda_err(e, "cudaGetSymbolAddress(status)");
+      nd.scratch = scratch;
+      nd.status = static_cast<int*>(status);
+      nd.ready = true;
+    }
+    local.status = nd.status;
+    local.checked = local.is_sm100 = true;
+    std::memcpy(local.bwd_attr, nd.bwd_attr, sizeof(local.bwd_attr));
+  }
+  // The first kernel of the backward rewrites every scratch byte the later ones read (dQ
+  // accumulator zeroed, D and -lse*log2e recomputed), so the previous call's contents do not
+  // matter.
+  st = bwd_dispatch(&local, q, k, v, o, dO, lse, dq, dk, dv, g_noalloc[dev].scratch, B * H, N, d,
+                    scale, causal != 0, static_cast<cudaStream_t>(stream));
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    std::memcpy(g_noalloc[dev].bwd_attr, local.bwd_attr, sizeof(local.bwd_attr));
+  }
+  return st;
 }
 
 fa_status fa_check_status(void* stream) {

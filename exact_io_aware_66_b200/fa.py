@@ -36,6 +36,7 @@ SIGNATURES = {
     "fa_profile_enable": (_I, [_I]),
     "fa_profile_read": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), _I]),
     "fa_kernel_name": (ctypes.c_char_p, [_I]),
+    "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
 }
 
 KERNEL_KINDS = 4
@@ -142,6 +143,24 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, causal: bool = False,
     st = lib().fa_bwd(*ptrs, workspace.data_ptr(), wbytes, B, H, N, d, scale, int(bool(causal)),
                       _stream_handle(stream))
     _check("fa_bwd", st)
+
+
+def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal: bool = False,
+                   scale: float | None = None, stream=None):
+    """Backward into caller-allocated dq, dk, dv with the library's built-in scratch instead of
+    a workspace, for callers that cannot allocate device memory (see include/fa.h: 64 MiB
+    limit; calls that overlap on the GPU race on the shared scratch)."""
+    B, H, N, d = _dims(q)
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (do, "do"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        if _dims(t) != (B, H, N, d):
+            raise ValueError(f"{n} shape mismatch")
+    if tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be [B, H, N]")
+    ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(do, "do"),
+            _req(lse, "lse", torch.float32), _req(dq, "dq"), _req(dk, "dk"), _req(dv, "dv")]
+    scale = default_scale(d) if scale is None else float(scale)
+    st = lib().fa_bwd_noalloc(*ptrs, B, H, N, d, scale, int(bool(causal)), _stream_handle(stream))
+    _check("fa_bwd_noalloc", st)
 
 
 def fa_profile_enable(on: bool = True):

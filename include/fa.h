@@ -71,6 +71,26 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
                  void* stream);
 
+/* Backward that allocates nothing (no counterpart in the paper: it exists for callers).
+ * Some callers cannot allocate device memory: a plugin running inside a framework that has
+ * reserved the GPU's memory for its own pool and hands out no workspace, or a service that
+ * must not allocate after start-up to keep its latency and memory footprint fixed. They call
+ * this instead of fa_bwd: same arguments without the workspace, same results.
+ * The scratch (fp32 dQ accumulator, per-row terms) is a 64 MiB array built into the library:
+ * every GPU that loads the library holds it until the process exits. Sizes whose
+ * fa_bwd_workspace_size exceeds 64 MiB (67108864 bytes) are rejected with FA_ERR_UNSUPPORTED
+ * and nothing is launched. This call performs no cudaMalloc, cudaFree or other allocation.
+ * Set-up: the first call on a device (with that device current) looks up the scratch's device
+ * address once; make that first call before any stream capture.
+ * All calls on a device share the one scratch array, which keeps the last call's contents (each
+ * call rewrites what it reads before reading it): calls that overlap on the GPU (different
+ * streams, or host threads, without ordering between them) race on it and must be serialised
+ * by the caller. A timed-out in-kernel wait (the hang guard) is recorded in a status word
+ * built into the library, not in the one fa_check_status reads. */
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const void* dO, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, float scale, int causal, void* stream);
+
 /* Synchronises `stream`, then reads and clears the current device's status word.
  * Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA. */
 fa_status fa_check_status(void* stream);
