@@ -376,51 +376,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t id_s = idesc_bf16_f32(128, 64, false, false);   // S^T, dP^T
       const uint32_t id_acc = idesc_bf16_f32(128, D, false, true);   // dV, dK
       const uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);    // dQ^T
+      // Operand descriptors are built once; per stage/buffer and k-step they are advanced by
+      // byte offsets (see sdesc_advance).
+      const uint64_t dK_k = sdesc_sw128(sbase + L::kK, 16, 1024);          // K, K-major
+      const uint64_t dV_k = sdesc_sw128(sbase + L::kV, 16, 1024);          // V, K-major
+      const uint64_t dKt_mn =                                              // K^T, MN-major
+          sdesc_sw128(sbase + L::kK, D == 128 ? static_cast<uint32_t>(L::kKVBox) : 0u, 1024);
+      const uint64_t dQ_k = sdesc_sw128(sbase + L::kQ, 16, 1024);          // Q, K-major
+      const uint64_t dDO_k = sdesc_sw128(sbase + L::kDO, 16, 1024);        // dO, K-major
+      const uint64_t dQ_mn = sdesc_sw128(sbase + L::kQ, L::kQBox, 1024);   // Q, MN-major
+      const uint64_t dDO_mn = sdesc_sw128(sbase + L::kDO, L::kQBox, 1024); // dO, MN-major
+      const uint64_t dDS = sdesc_sw128(sbase + L::kDS, 16, 1024);          // dS^T (K- or MN-major)
       auto first_half = [&](int i) {
-        const int b = i & 1, st = i % QS;
-        const uint32_t qa = sbase + L::kQ + st * 2 * L::kQTile;
-        const uint32_t da = sbase + L::kDO + st * 2 * L::kQTile;
+        const int b = i & 1;
+        const uint32_t so = static_cast<uint32_t>(i % QS) * 2 * L::kQTile;
+        const uint64_t q0 = sdesc_advance(dQ_k, so), o0 = sdesc_advance(dDO_k, so);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t okv = (kk >> 2) * L::kKVBox + (kk & 3) * 32;
           const uint32_t oq = (kk >> 2) * L::kQBox + (kk & 3) * 32;
-          umma_ss(tmem + L::tS(b), sdesc_sw128(sbase + L::kK + okv, 16, 1024),
-                  sdesc_sw128(qa + oq, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + L::tS(b), sdesc_advance(dK_k, okv), sdesc_advance(q0, oq), id_s,
+                  kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t okv = (kk >> 2) * L::kKVBox + (kk & 3) * 32;
           const uint32_t oq = (kk >> 2) * L::kQBox + (kk & 3) * 32;
-          umma_ss(tmem + L::tDP(b), sdesc_sw128(sbase + L::kV + okv, 16, 1024),
-                  sdesc_sw128(da + oq, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + L::tDP(b), sdesc_advance(dV_k, okv), sdesc_advance(o0, oq), id_s,
+                  kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(L::bSdPFull + b));
       };
       auto second_half = [&](int i) {
         const int b = i & 1, st = i % QS;
-        const uint32_t qa = sbase + L::kQ + st * 2 * L::kQTile;
-        const uint32_t da = sbase + L::kDO + st * 2 * L::kQTile;
-        const uint32_t dsa = sbase + L::kDS + b * 16384;
+        const uint32_t so = static_cast<uint32_t>(st) * 2 * L::kQTile;
+        const uint64_t qmn = sdesc_advance(dQ_mn, so), omn = sdesc_advance(dDO_mn, so);
+        const uint64_t ds = sdesc_advance(dDS, b * 16384);
+        const uint32_t acc = i > 0 ? 1u : 0u;
         // dV += P^T dO: P^T (keys x 64 queries) from TMEM; query columns 0-31 were packed into
         // S columns [0,16), 32-63 into [32,48).
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_ts(tmem + L::tDV, tmem + L::tS(b) + (kk >> 1) * 32 + (kk & 1) * 8,
-                  sdesc_sw128(da + kk * 2048, L::kQBox, 1024), id_acc,
-                  (i > 0 || kk > 0) ? 1u : 0u);
+                  sdesc_advance(omn, kk * 2048), id_acc, kk > 0 ? 1u : acc);
         // dK += dS^T Q
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_ss(tmem + L::tDK, sdesc_sw128(dsa + kk * 32, 16, 1024),
-                  sdesc_sw128(qa + kk * 2048, L::kQBox, 1024), id_acc,
-                  (i > 0 || kk > 0) ? 1u : 0u);
+          umma_ss(tmem + L::tDK, sdesc_advance(ds, kk * 32), sdesc_advance(qmn, kk * 2048), id_acc,
+                  kk > 0 ? 1u : acc);
         // dQ^T = K^T dS^T  (M = 128 rows of d; for d = 64 the second half of the rows repeats
         // the first and is ignored by the drain)
-        const uint32_t lbo_k = D == 128 ? static_cast<uint32_t>(L::kKVBox) : 0u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + L::tDP(b), sdesc_sw128(sbase + L::kK + kk * 2048, lbo_k, 1024),
-                  sdesc_sw128(dsa + kk * 2048, 16, 1024), id_dq, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + L::tDP(b), sdesc_advance(dKt_mn, kk * 2048), sdesc_advance(ds, kk * 2048),
+                  id_dq, kk > 0 ? 1u : 0u);
         umma_commit(bar(L::bDQFull + b));
         umma_commit(bar(L::bQEmpty + st));
         umma_commit(bar(L::bDSFree + b));

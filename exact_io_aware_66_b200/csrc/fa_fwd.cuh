@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       p.lse[static_cast<size_t>(bh) * p.N + q_row] = (m * sl2 + lg2_approx(l)) * 0.69314718055994531f;
   } else if (warp < 12) {
     // ----------------------------------------------------------------- epilogue ----------
-    setmaxnreg_dec<80>();
+    setmaxnreg_dec<64>();
     const int row = threadIdx.x - 256;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
@@ -313,35 +313,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     if (lane == 0) bulk_wait_group_read0();
   } else {
-    setmaxnreg_dec<80>();
+    setmaxnreg_dec<96>();
     if (warp == 12 && lane == 0) {
       // ------------------------------------------------------------------ MMA -------------
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      auto stage_addr = [&](int tt) -> uint32_t {
-        return sbase + L::kKV + static_cast<uint32_t>(tt % ST) * L::kTileBytes;
-      };
+      // Operand descriptors are built once; per k-step they are advanced by constant offsets.
+      const uint64_t desc_q0 = sdesc_sw128(sbase + L::kQ, 16, 1024);             // K-major
+      const uint64_t desc_k0 = sdesc_sw128(sbase + L::kKV, 16, 1024);            // K-major
+      const uint64_t desc_v0 = sdesc_sw128(sbase + L::kKV, L::kBoxBytes, 1024);  // MN-major
       auto wait_full = [&](int tt) -> bool {
         return mbar_wait(bar(L::bKvFull + tt % ST), (tt / ST) & 1, abort_flag);
       };
       auto issue_s = [&](int t, int j) {
-        const uint32_t qa = sbase + L::kQ + t * L::kTileBytes;
-        const uint32_t ka = stage_addr(2 * j);
+        const uint64_t a0 = sdesc_advance(desc_q0, t * L::kTileBytes);
+        const uint64_t b0 = sdesc_advance(desc_k0, ((2 * j) % ST) * L::kTileBytes);
+        const uint32_t d = tmem + t * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          umma_ss(tmem + t * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
-                  idesc_qk, kk > 0 ? 1u : 0u);
+          umma_ss(d, sdesc_advance(a0, off), sdesc_advance(b0, off), idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(L::bSFull + t));
       };
       auto issue_pv = [&](int t, int j) {
-        const uint32_t va = stage_addr(2 * j + 1);
+        const uint64_t b0 = sdesc_advance(desc_v0, ((2 * j + 1) % ST) * L::kTileBytes);
+        const uint32_t d = tmem + 256 + t * D, a = tmem + t * 128;
+        umma_ts(d, a, b0, idesc_pv, j > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
-                  sdesc_sw128(va + kk * 2048, L::kBoxBytes, 1024), idesc_pv,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 1; kk < 8; ++kk)
+          umma_ts(d, a + kk * 8, sdesc_advance(b0, kk * 2048), idesc_pv, 1u);
         umma_commit(bar(L::bODone + t));
       };
       bool ok = mbar_wait(bar(L::bQ), 0, abort_flag) && wait_full(0);
