@@ -202,6 +202,14 @@ fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* 
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return cuda_err(e, "cudaFuncSetAttribute(fwd smem)");
+    // The kernel redistributes registers with setmaxnreg, whose split assumes 128 per thread
+    // at launch; any other allocation could make setmaxnreg.inc wait forever.
+    cudaFuncAttributes fattr;
+    e = cudaFuncGetAttributes(&fattr, kern);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncGetAttributes(fwd)");
+    if (fattr.numRegs != 128)
+      return set_err(FA_ERR_CUDA, "forward kernel built with %d registers per thread, 128 expected",
+                     fattr.numRegs);
     attr = true;
   }
   CUtensorMap tq, tk, tv, to;
@@ -325,6 +333,21 @@ fa_status bwd_dispatch(DeviceState* ds, const void* q, const void* k, const void
                   : launch_bwd<64, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream);
   return causal ? launch_bwd<128, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream)
                 : launch_bwd<128, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream);
+}
+
+// ---- failure-detection self-test ----
+// One thread waits, through the same bounded mbar_wait the attention kernels use, on an mbarrier
+// that nothing ever arrives at. The wait gives up after `limit_ns`, the kernel records
+// FA_ERR_TIMEOUT in the status word exactly as a timed-out attention kernel does, and returns.
+__global__ void fa_selftest_timeout_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long bar_storage;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  const uint32_t bar = fa::smem_u32(&bar_storage);
+  fa::mbar_init(bar, 1);
+  fa::fence_barrier_init();
+  if (!fa::mbar_wait(bar, 0, &abort_flag, limit_ns)) atomicExch(status, FA_ERR_TIMEOUT);
 }
 
 // ---- fa_bwd_noalloc: backward whose scratch is built into the library ----
@@ -523,6 +546,20 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
     std::memcpy(g_noalloc[dev].bwd_attr, local.bwd_attr, sizeof(local.bwd_attr));
   }
   return st;
+}
+
+fa_status fa_selftest_timeout(int limit_us, void* stream) {
+  g_err[0] = '\0';
+  if (limit_us < 1 || limit_us > 10000000)
+    return set_err(FA_ERR_INVALID_ARG, "limit_us must be in [1, 10^7] (got %d)", limit_us);
+  fa_status st;
+  DeviceState* ds = device_state(&st);
+  if (!ds) return st;
+  fa_selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      ds->status, 1000ull * static_cast<unsigned long long>(limit_us));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_selftest_timeout launch");
+  return FA_OK;
 }
 
 fa_status fa_check_status(void* stream) {

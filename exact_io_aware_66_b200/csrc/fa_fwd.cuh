@@ -27,6 +27,12 @@
 namespace fa {
 
 constexpr int kFwdThreads = 512;
+// Register split (setmaxnreg): softmax warps 0-7, epilogue warps 8-11, MMA/TMA warps 12-15.
+// setmaxnreg.inc waits until the decrements have freed enough registers, so the split must add
+// up to exactly the launch allocation (512 threads x 128 registers; checked on the host).
+constexpr uint32_t kFwdRegSoftmax = 176, kFwdRegEpilogue = 64, kFwdRegMma = 96;
+static_assert(256 * kFwdRegSoftmax + 128 * kFwdRegEpilogue + 128 * kFwdRegMma == kFwdThreads * 128,
+              "forward register split must equal the launch allocation");
 // Running-max update threshold, log2 units (exponentials stay below 2^8 between updates).
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -159,7 +165,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (warp < 8) {
     // ------------------------------------------------------------------ softmax ----------
-    setmaxnreg_inc<176>();
+    setmaxnreg_inc<kFwdRegSoftmax>();
     const int t = warp >> 2;
     const int row = threadIdx.x & 127;
     const uint32_t tS = tmem + t * 128 + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -265,7 +271,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       p.lse[static_cast<size_t>(bh) * p.N + q_row] = (m * sl2 + lg2_approx(l)) * 0.69314718055994531f;
   } else if (warp < 12) {
     // ----------------------------------------------------------------- epilogue ----------
-    setmaxnreg_dec<64>();
+    setmaxnreg_dec<kFwdRegEpilogue>();
     const int row = threadIdx.x - 256;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
@@ -313,7 +319,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     if (lane == 0) bulk_wait_group_read0();
   } else {
-    setmaxnreg_dec<96>();
+    setmaxnreg_dec<kFwdRegMma>();
     if (warp == 12 && lane == 0) {
       // ------------------------------------------------------------------ MMA -------------
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);

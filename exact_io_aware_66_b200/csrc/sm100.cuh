@@ -59,17 +59,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for phase `parity` of `bar` to complete. Returns false when the time limit
-// expires or when *abort becomes non-zero (another role of the CTA gave up); never spins
-// forever.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+// Bounded wait for phase `parity` of `bar` to complete. Returns false when `limit_ns`
+// nanoseconds pass or when *abort becomes non-zero (another role of the CTA gave up); never
+// spins forever.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = FA_SPIN_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > FA_SPIN_LIMIT_NS) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
     }
   }
 }

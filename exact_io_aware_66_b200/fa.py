@@ -37,6 +37,7 @@ SIGNATURES = {
     "fa_profile_read": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), _I]),
     "fa_kernel_name": (ctypes.c_char_p, [_I]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_selftest_timeout": (_I, [_I, _P]),
 }
 
 KERNEL_KINDS = 4
@@ -174,6 +175,12 @@ def fa_profile_read() -> dict:
     _check("fa_profile_read", lib().fa_profile_read(ms, n, KERNEL_KINDS))
     return {lib().fa_kernel_name(i).decode(): (int(n[i]), float(ms[i]))
             for i in range(KERNEL_KINDS)}
+
+
+def fa_selftest_timeout(limit_us: int = 20000, stream=None):
+    """Launches the bounded-wait self-test kernel (see include/fa.h); follow with
+    fa_check_status(), which must then raise FaError with FA_ERR_TIMEOUT."""
+    _check("fa_selftest_timeout", lib().fa_selftest_timeout(int(limit_us), _stream_handle(stream)))
 
 
 def fa_check_status(stream=None):

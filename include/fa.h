@@ -91,6 +91,13 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          const void* dO, const float* lse, void* dq, void* dk, void* dv, int B,
                          int H, int N, int d, float scale, int causal, void* stream);
 
+/* Failure-detection self-test: launches on `stream` a one-thread kernel that waits, through the
+ * same bounded wait the attention kernels use, on a barrier nothing ever completes. After
+ * limit_us microseconds (1 .. 10^7) the wait gives up, FA_ERR_TIMEOUT is recorded in the
+ * device status word and the kernel returns; the GPU is neither faulted nor hung. A following
+ * fa_check_status(stream) returns FA_ERR_TIMEOUT and clears the word. */
+fa_status fa_selftest_timeout(int limit_us, void* stream);
+
 /* Synchronises `stream`, then reads and clears the current device's status word.
  * Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA. */
 fa_status fa_check_status(void* stream);

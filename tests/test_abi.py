@@ -112,3 +112,8 @@ def test_no_cpu_fallback_in_product_package():
         if fn.endswith(".py"):
             src = open(os.path.join(pkg, fn)).read()
             assert not re.search(r"^\s*(from|import)\s+oracle", src, flags=re.M), fn
+
+
+def test_selftest_timeout_rejects_bad_limit_without_gpu(lib):
+    assert lib.fa_selftest_timeout(0, None) == 1
+    assert lib.fa_selftest_timeout(10 ** 8, None) == 1
