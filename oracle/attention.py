@@ -17,9 +17,15 @@ What is computed, and where it is defined:
       lse_i = m_i + ln l_i                      (natural log; the stored "normalization
                                                  factors" of "Backward Pass Recomputation")
   The max subtraction changes nothing mathematically; it keeps exp() in range.
-* Causal masking (key j visible to query i iff j <= i, square, top-left aligned): masked
-  entries are left out of every sum, i.e. they contribute exactly zero. The pages name masking
-  only as one of standard attention's HBM passes ("The GPU Memory Wall: HBM vs. SRAM").
+* Causal masking: masked entries are left out of every sum, i.e. they contribute exactly zero.
+  The pages name masking only as one of standard attention's HBM passes ("The GPU Memory Wall:
+  HBM vs. SRAM"). Modes: "none"; "top_left" (key j visible to query i iff j <= i; also
+  `causal=True`); "bottom_right" (iff j <= i + N_k - N_q, the alignment where the last query
+  sees every key, as in decoding). A query row that sees no key at all (bottom-right with
+  N_q > N_k) has O = 0 and lse = -inf, and contributes nothing to any gradient.
+* Grouped heads: when K and V have H_kv < H heads ([B, H_kv, N_k, d] against [B, H, N_q, d],
+  H a multiple of H_kv), query head h uses key/value head h // (H / H_kv); the gradients of a
+  key/value head sum over the query heads that share it.
 * Backward. The pages say only that the scores are recomputed on chip and the gradients
   calculated ("The Backward Pass: Recomputation"). The formulas are the calculus of the
   definition above, with P_ij = exp(s_ij - lse_i) and L a scalar loss with dO = dL/dO:
@@ -63,15 +69,37 @@ def _f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def _visible(i: int, n_keys: int, causal: bool) -> int:
-    """Number of keys visible to query row i (keys 0 .. result-1)."""
-    return min(i + 1, n_keys) if causal else n_keys
+def _mode(causal) -> str:
+    """Normalises the mask argument: False/None/"none", True/"top_left", "bottom_right"."""
+    if causal is True:
+        return "top_left"
+    if causal is False or causal is None:
+        return "none"
+    if causal in ("none", "top_left", "bottom_right"):
+        return causal
+    raise ValueError(f"unknown mask mode {causal!r}")
+
+
+def _visible(i: int, n_q: int, n_keys: int, mode: str) -> int:
+    """Number of keys visible to query row i (keys 0 .. result-1); may be 0."""
+    if mode == "none":
+        return n_keys
+    off = (n_keys - n_q) if mode == "bottom_right" else 0
+    return int(min(max(i + 1 + off, 0), n_keys))
 
 
 def _head_iter(shape):
     """Iterate over every leading index of a [..., N, d] array."""
     lead = shape[:-2]
     return np.ndindex(*lead) if lead else iter([()])
+
+
+def _kv_index(idx, q_shape, k_shape):
+    """Leading index of the key/value head used by the query head at leading index `idx`."""
+    if len(q_shape) >= 4 and k_shape[-3] != q_shape[-3]:
+        group = q_shape[-3] // k_shape[-3]
+        return tuple(idx[:-1]) + (idx[-1] // group,)
+    return idx
 
 
 def _softmax_block(s: np.ndarray, mask: np.ndarray | None):
@@ -85,54 +113,71 @@ def _softmax_block(s: np.ndarray, mask: np.ndarray | None):
         e = np.exp(s - m[:, None])
     else:
         m = np.where(mask, s, -np.inf).max(axis=1)
-        e = np.where(mask, np.exp(np.where(mask, s, 0.0) - m[:, None]), 0.0)
+        m_safe = np.where(np.isfinite(m), m, 0.0)  # rows without any visible key
+        e = np.where(mask, np.exp(np.where(mask, s, 0.0) - m_safe[:, None]), 0.0)
     return m, e, e.sum(axis=1)
 
 
-def _causal_mask(r0: int, r1: int, n_keys: int) -> np.ndarray:
+def _finish(e, l, m, v):
+    """O = e V / l and lse = m + ln l, with O = 0 and lse = -inf for rows that see no key."""
+    empty = l == 0.0
+    o = (e @ v) / np.where(empty, 1.0, l)[:, None]
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty, -np.inf, m + np.log(np.where(empty, 1.0, l)))
+    return o, lse
+
+
+def _mask(r0: int, r1: int, n_q: int, n_keys: int, mode: str):
+    """Visibility of keys [0, n_keys) to query rows [r0, r1), or None when all are visible."""
+    if mode == "none":
+        return None
+    off = (n_keys - n_q) if mode == "bottom_right" else 0
     rows = np.arange(r0, r1)[:, None]
     cols = np.arange(n_keys)[None, :]
-    return cols <= rows
+    return cols <= rows + off
 
 
-def attention_probabilities(q, k, scale: float, causal: bool = False) -> np.ndarray:
+def attention_probabilities(q, k, scale: float, causal=False) -> np.ndarray:
     """P = softmax(scale * Q K^T) per the definition (codethepapers.com, "The Problem: The
-    Memory Wall"), masked entries exactly 0. Shapes: q [..., N, d], k [..., M, d] ->
-    [..., N, M]. Small inputs only (materialises N x M)."""
+    Memory Wall"), masked entries exactly 0 (rows that see no key are all 0). Shapes:
+    q [..., N, d], k [..., M, d] -> [..., N, M]. Small inputs only (materialises N x M)."""
     q, k = _f64(q), _f64(k)
+    mode = _mode(causal)
     scale = float(np.float64(scale))
     out = np.zeros(q.shape[:-1] + (k.shape[-2],), dtype=np.float64)
     for idx in _head_iter(q.shape):
-        s = scale * (q[idx] @ k[idx].T)
-        mask = _causal_mask(0, q.shape[-2], k.shape[-2]) if causal else None
-        _, e, l = _softmax_block(s, mask)
-        out[idx] = e / l[:, None]
+        kh = k[_kv_index(idx, q.shape, k.shape)]
+        s = scale * (q[idx] @ kh.T)
+        _, e, l = _softmax_block(s, _mask(0, q.shape[-2], q.shape[-2], k.shape[-2], mode))
+        out[idx] = e / np.where(l == 0.0, 1.0, l)[:, None]
     return out
 
 
-def attention_forward(q, k, v, scale: float, causal: bool = False, block_rows: int = 512):
-    """Exact attention forward: returns (O [..., N, d], lse [..., N]) in float64.
+def attention_forward(q, k, v, scale: float, causal=False, block_rows: int = 512):
+    """Exact attention forward: returns (O [..., N_q, d], lse [..., N_q]) in float64.
 
     Definition: codethepapers.com, "The Problem: The Memory Wall" (P = softmax(QK^T/sqrt d),
     output P V) with the running max m and sum l of hot.atechcom.net, "The Secret Weapon:
-    Online Softmax"; lse = m + ln l. Masked entries (causal, j > i) contribute exactly 0.
+    Online Softmax"; lse = m + ln l. Masked entries contribute exactly 0; `causal` is a mask
+    mode (see the module docstring); K/V may have fewer heads than Q (grouped heads).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
+    mode = _mode(causal)
     scale = float(np.float64(scale))
     n, nk = q.shape[-2], k.shape[-2]
     o = np.zeros(q.shape[:-1] + (v.shape[-1],), dtype=np.float64)
     lse = np.zeros(q.shape[:-1], dtype=np.float64)
     for idx in _head_iter(q.shape):
-        qh, kh, vh = q[idx], k[idx], v[idx]
+        kvi = _kv_index(idx, q.shape, k.shape)
+        qh, kh, vh = q[idx], k[kvi], v[kvi]
         for r0 in range(0, n, block_rows):
             r1 = min(n, r0 + block_rows)
             # keys beyond the last visible one of this block are masked for every row in it
-            kv_end = _visible(r1 - 1, nk, causal)
+            kv_end = _visible(r1 - 1, n, nk, mode)
             s = scale * (qh[r0:r1] @ kh[:kv_end].T)
-            mask = _causal_mask(r0, r1, kv_end) if causal else None
-            m, e, l = _softmax_block(s, mask)
-            o[idx][r0:r1] = (e @ vh[:kv_end]) / l[:, None]
-            lse[idx][r0:r1] = m + np.log(l)
+            m, e, l = _softmax_block(s, _mask(r0, r1, n, nk, mode)[:, :kv_end]
+                                     if mode != "none" else None)
+            o[idx][r0:r1], lse[idx][r0:r1] = _finish(e, l, m, vh[:kv_end])
     return o, lse
 
 
@@ -147,27 +192,33 @@ def attention_backward(q, k, v, do, scale: float, causal: bool = False, block_ro
     Actually Works", "The Backward Pass: Recomputation"). D uses the oracle's own fp64 O.
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    mode = _mode(causal)
     scale = float(np.float64(scale))
-    o, lse = attention_forward(q, k, v, scale, causal, block_rows)
+    o, lse = attention_forward(q, k, v, scale, mode, block_rows)
     n, nk = q.shape[-2], k.shape[-2]
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     for idx in _head_iter(q.shape):
-        qh, kh, vh, doh = q[idx], k[idx], v[idx], do[idx]
+        kvi = _kv_index(idx, q.shape, k.shape)
+        qh, kh, vh, doh = q[idx], k[kvi], v[kvi], do[idx]
         dd = np.sum(doh * o[idx], axis=1)  # D_i
         for r0 in range(0, n, block_rows):
             r1 = min(n, r0 + block_rows)
-            kv_end = _visible(r1 - 1, nk, causal)
+            kv_end = _visible(r1 - 1, n, nk, mode)
+            if kv_end == 0:
+                continue  # no row of this block sees a key: no gradient flows
             s = scale * (qh[r0:r1] @ kh[:kv_end].T)
-            p = np.exp(s - lse[idx][r0:r1, None])
-            if causal:
-                p = np.where(_causal_mask(r0, r1, kv_end), p, 0.0)
-            dv[idx][:kv_end] += p.T @ doh[r0:r1]
+            mask = _mask(r0, r1, n, nk, mode)
+            with np.errstate(over="ignore"):
+                p = np.exp(s - lse[idx][r0:r1, None])
+            if mask is not None:
+                p = np.where(mask[:, :kv_end], p, 0.0)
+            dv[kvi][:kv_end] += p.T @ doh[r0:r1]
             dp = doh[r0:r1] @ vh[:kv_end].T
             ds = p * (dp - dd[r0:r1, None])
             dq[idx][r0:r1] = scale * (ds @ kh[:kv_end])
-            dk[idx][:kv_end] += scale * (ds.T @ qh[r0:r1])
+            dk[kvi][:kv_end] += scale * (ds.T @ qh[r0:r1])
     if return_forward:
         return dq, dk, dv, o, lse
     return dq, dk, dv
@@ -182,16 +233,21 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, do=None):
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     do = None if do is None else _f64(do)
+    mode = _mode(causal)
     scale = float(np.float64(scale))
     rows = [tuple(int(t) for t in r) for r in rows]
-    nk = k.shape[-2]
+    n, nk = q.shape[-2], k.shape[-2]
     o_out = np.zeros((len(rows), v.shape[-1]))
     lse_out = np.zeros(len(rows))
     dq_out = np.zeros((len(rows), q.shape[-1])) if do is not None else None
     for t, r in enumerate(rows):
         head, i = r[:-1], r[-1]
-        vis = _visible(i, nk, causal)
-        kh, vh = k[head][:vis], v[head][:vis]
+        vis = _visible(i, n, nk, mode)
+        if vis == 0:
+            lse_out[t] = -np.inf  # O and dQ stay 0
+            continue
+        kvi = _kv_index(head, q.shape, k.shape)
+        kh, vh = k[kvi][:vis], v[kvi][:vis]
         s = scale * (kh @ q[head][i])
         m = s.max()
         e = np.exp(s - m)
@@ -210,30 +266,42 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, do=None):
     return o_out, lse_out
 
 
-def attention_keys(q, k, v, do, scale: float, causal: bool, head, keys, block_rows: int = 512):
-    """dK and dV rows for selected keys j of one head (leading index tuple `head`).
+def attention_keys(q, k, v, do, scale: float, causal, head, keys, block_rows: int = 512):
+    """dK and dV rows for selected keys j of one key/value head (leading index tuple `head`,
+    e.g. (b, h_kv)).
 
-    dV_j = sum_i P_ij dO_i and dK_j = scale sum_i dS_ij q_i over the query rows that see key j.
-    Needs lse_i and D_i of every row of the head, so the head's full forward is computed first.
-    Returns (dK_rows [n, d], dV_rows [n, d]).
+    dV_j = sum_i P_ij dO_i and dK_j = scale sum_i dS_ij q_i over the query rows that see key j,
+    in every query head that uses this key/value head. Needs lse_i and D_i of those rows, so
+    their full forward is computed first. Returns (dK_rows [n, d], dV_rows [n, d]).
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    mode = _mode(causal)
     scale = float(np.float64(scale))
     head = tuple(int(t) for t in head)
-    qh, kh, vh, doh = q[head], k[head], v[head], do[head]
-    o, lse = attention_forward(qh, kh, vh, scale, causal, block_rows)
-    dd = np.sum(doh * o, axis=1)
-    n = qh.shape[0]
+    kh, vh = k[head], v[head]
+    n, nk = q.shape[-2], k.shape[-2]
+    if q.ndim >= 4 and k.shape[-3] != q.shape[-3]:
+        group = q.shape[-3] // k.shape[-3]
+        q_heads = [head[:-1] + (head[-1] * group + g,) for g in range(group)]
+    else:
+        q_heads = [head]
+    off = (nk - n) if mode == "bottom_right" else 0
     dk_out = np.zeros((len(keys), kh.shape[1]))
     dv_out = np.zeros((len(keys), vh.shape[1]))
-    for t, j in enumerate(int(x) for x in keys):
-        i0 = j if causal else 0  # rows i >= j see key j under the causal mask
-        s = scale * (qh[i0:n] @ kh[j])
-        p = np.exp(s - lse[i0:n])
-        dv_out[t] = p @ doh[i0:n]
-        dp = doh[i0:n] @ vh[j]
-        ds = p * (dp - dd[i0:n])
-        dk_out[t] = scale * (ds @ qh[i0:n])
+    for qh_idx in q_heads:
+        qh, doh = q[qh_idx], do[qh_idx]
+        o, lse = attention_forward(qh, kh, vh, scale, mode, block_rows)
+        dd = np.sum(doh * o, axis=1)
+        for t, j in enumerate(int(x) for x in keys):
+            i0 = 0 if mode == "none" else max(0, j - off)  # rows i with j <= i + off see key j
+            if i0 >= n:
+                continue
+            s = scale * (qh[i0:n] @ kh[j])
+            p = np.exp(s - lse[i0:n])
+            dv_out[t] += p @ doh[i0:n]
+            dp = doh[i0:n] @ vh[j]
+            ds = p * (dp - dd[i0:n])
+            dk_out[t] += scale * (ds @ qh[i0:n])
     return dk_out, dv_out
 
 
