@@ -181,20 +181,40 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
-fa_status check_sizes(int B, int H, int N, int d, float scale) {
-  if (B < 1 || H < 1 || N < 1)
-    return set_err(FA_ERR_INVALID_ARG, "B, H, N must be >= 1 (got %d, %d, %d)", B, H, N);
-  if (d != 64 && d != 128) return set_err(FA_ERR_UNSUPPORTED, "head dim d=%d not in {64, 128}", d);
-  const long long rows = 1LL * B * H * N;
-  if (rows >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "B*H*N=%lld >= 2^31", rows);
-  if (!std::isfinite(scale) || !(scale > 0.f))
-    return set_err(FA_ERR_INVALID_ARG, "scale must be finite and > 0 (got %g)", (double)scale);
+// Problem shape shared by every entry point: q, o, dO, dq are [B, H, N_q, d]; k, v, dk, dv are
+// [B, H_kv, N_kv, d]; lse is [B, H, N_q]. mask: 0 none, 1 causal aligned at the top left
+// (key j visible to query i iff j <= i), 2 causal aligned at the bottom right (iff
+// j <= i + N_kv - N_q).
+struct Shape {
+  int B, H, H_kv, N_q, N_kv, d;
+  float scale;
+  int mask;
+  size_t q_bytes() const { return static_cast<size_t>(B) * H * N_q * d * 2; }
+  size_t kv_bytes() const { return static_cast<size_t>(B) * H_kv * N_kv * d * 2; }
+  size_t lse_bytes() const { return static_cast<size_t>(B) * H * N_q * 4; }
+  int off() const { return mask == 2 ? N_kv - N_q : 0; }
+};
+
+fa_status check_shape(const Shape& s) {
+  if (s.B < 1 || s.H < 1 || s.H_kv < 1 || s.N_q < 1 || s.N_kv < 1)
+    return set_err(FA_ERR_INVALID_ARG, "B, H, H_kv, N_q, N_kv must be >= 1 (got %d, %d, %d, %d, %d)",
+                   s.B, s.H, s.H_kv, s.N_q, s.N_kv);
+  if (s.H % s.H_kv != 0)
+    return set_err(FA_ERR_INVALID_ARG, "H=%d is not a multiple of H_kv=%d", s.H, s.H_kv);
+  if (s.d != 64 && s.d != 128)
+    return set_err(FA_ERR_UNSUPPORTED, "head dim d=%d not in {64, 128}", s.d);
+  if (s.mask < 0 || s.mask > 2) return set_err(FA_ERR_INVALID_ARG, "mask mode %d unknown", s.mask);
+  const long long rows_q = 1LL * s.B * s.H * s.N_q, rows_kv = 1LL * s.B * s.H_kv * s.N_kv;
+  if (rows_q >= (1LL << 31) || rows_kv >= (1LL << 31))
+    return set_err(FA_ERR_UNSUPPORTED, "B*H*N_q=%lld or B*H_kv*N_kv=%lld >= 2^31", rows_q, rows_kv);
+  if (!std::isfinite(s.scale) || !(s.scale > 0.f))
+    return set_err(FA_ERR_INVALID_ARG, "scale must be finite and > 0 (got %g)", (double)s.scale);
   return FA_OK;
 }
 
 template <int D, bool CAUSAL>
 fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
-                     float* lse, int BH, int N, float scale, cudaStream_t stream) {
+                     float* lse, const Shape& s, cudaStream_t stream) {
   using L = fa::FwdLayout<D>;
   auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
   bool& attr = ds->fwd_attr[D == 128][CAUSAL];
@@ -212,20 +232,24 @@ fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* 
                      fattr.numRegs);
     attr = true;
   }
+  const int BH = s.B * s.H, BHkv = s.B * s.H_kv;
   CUtensorMap tq, tk, tv, to;
   fa_status st;
-  if ((st = make_bf16_map(&tq, q, D, N, BH, 128)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tk, k, D, N, BH, 128)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tv, v, D, N, BH, 128)) != FA_OK) return st;
-  if ((st = make_bf16_map(&to, o, D, N, BH, 32)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tq, q, D, s.N_q, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tk, k, D, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tv, v, D, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&to, o, D, s.N_q, BH, 32)) != FA_OK) return st;
   fa::FwdParams p;
   p.lse = lse;
   p.status = ds->status;
-  p.N = N;
+  p.N = s.N_q;
+  p.N_kv = s.N_kv;
   p.BH = BH;
-  p.n_qblocks = (N + 255) / 256;
-  p.scale = scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.group = s.H / s.H_kv;
+  p.off = s.off();
+  p.n_qblocks = (s.N_q + 255) / 256;
+  p.scale = s.scale;
+  p.scale_log2 = s.scale * 1.4426950408889634f;
   const long long grid = 1LL * p.n_qblocks * BH;
   if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
   ProfileScope prof(0, stream);
@@ -238,7 +262,7 @@ fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* 
 template <int D, bool CAUSAL>
 fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* v, const void* o,
                      const void* dO, const float* lse, void* dq, void* dk, void* dv,
-                     void* workspace, int BH, int N, float scale, cudaStream_t stream) {
+                     void* workspace, const Shape& s, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
   auto kern = fa::fa_bwd_main<D, CAUSAL>;
   bool& attr = ds->bwd_attr[D == 128][CAUSAL];
@@ -248,6 +272,7 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
     if (e != cudaSuccess) return cuda_err(e, "cudaFuncSetAttribute(bwd smem)");
     attr = true;
   }
+  const int BH = s.B * s.H, BHkv = s.B * s.H_kv, N = s.N_q;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(ws);
   float* Dvec = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_D(BH, N, D));
@@ -258,19 +283,19 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   CUtensorMap tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv;
   fa_status st;
   if ((st = make_bf16_map(&tq, q, D, N, BH, 64)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tk, k, D, N, BH, 128)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tv, v, D, N, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tk, k, D, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tv, v, D, s.N_kv, BHkv, 128)) != FA_OK) return st;
   if ((st = make_bf16_map(&tdo, dO, D, N, BH, 64)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tdk, dk, D, N, BH, 32)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tdv, dv, D, N, BH, 32)) != FA_OK) return st;
-  // per-row fp32 vectors: [BH][N] with a row stride of N64 elements, 64-element boxes
+  if ((st = make_bf16_map(&tdk, dk, D, s.N_kv, BHkv, 32)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdv, dv, D, s.N_kv, BHkv, 32)) != FA_OK) return st;
+  // per-row fp32 vectors: [BH][N_q] with a row stride of N64 elements, 64-element boxes
   if ((st = make_map(&tl, lse2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 64, 1,
                      CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
     return st;
   if ((st = make_map(&tD, Dvec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 64, 1,
                      CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
     return st;
-  // dQ accumulator: fp32 [BH][N][D], reduction boxes of 32 columns x 64 rows
+  // dQ accumulator: fp32 [BH][N_q][D], reduction boxes of 32 columns x 64 rows
   if ((st = make_map(&tacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, 32, 64,
                      CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
     return st;
@@ -291,19 +316,23 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   fa::BwdParams p;
   p.status = ds->status;
   p.N = N;
-  p.BH = BH;
-  p.n_kv = (N + 127) / 128;
+  p.N_kv = s.N_kv;
+  p.BH_kv = BHkv;
+  p.qgroup = s.H / s.H_kv;
+  p.off = s.off();
+  p.n_kv = (s.N_kv + 127) / 128;
   p.n_q = (N + 63) / 64;
   {
-    // heads per scheduling group: Q, dO, K, V (bf16) and the fp32 dQ accumulator of a group
-    // should stay within about half of the 126 MB L2
-    const double per_head = static_cast<double>(N) * D * (2 + 2 + 2 + 2 + 4);
+    // key/value heads per scheduling group: a group's K, V, and its query heads' Q, dO (bf16)
+    // and fp32 dQ accumulator should stay within about half of the 126 MB L2
+    const double per_head = static_cast<double>(s.N_kv) * D * 4 +
+                            static_cast<double>(p.qgroup) * N * D * (2 + 2 + 4);
     const int g = static_cast<int>(64.0 * 1024 * 1024 / per_head);
-    p.group = g < 1 ? 1 : (g > BH ? BH : g);
+    p.group = g < 1 ? 1 : (g > BHkv ? BHkv : g);
   }
-  p.scale = scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  const long long grid = 1LL * p.n_kv * BH;
+  p.scale = s.scale;
+  p.scale_log2 = s.scale * 1.4426950408889634f;
+  const long long grid = 1LL * p.n_kv * BHkv;
   if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
   {
     ProfileScope prof(2, stream);
@@ -324,15 +353,87 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   return FA_OK;
 }
 
+fa_status fwd_dispatch(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
+                       float* lse, const Shape& s, cudaStream_t stream) {
+  const bool causal = s.mask != 0;
+  if (s.d == 64)
+    return causal ? launch_fwd<64, true>(ds, q, k, v, o, lse, s, stream)
+                  : launch_fwd<64, false>(ds, q, k, v, o, lse, s, stream);
+  return causal ? launch_fwd<128, true>(ds, q, k, v, o, lse, s, stream)
+                : launch_fwd<128, false>(ds, q, k, v, o, lse, s, stream);
+}
+
 fa_status bwd_dispatch(DeviceState* ds, const void* q, const void* k, const void* v, const void* o,
                        const void* dO, const float* lse, void* dq, void* dk, void* dv,
-                       void* workspace, int BH, int N, int d, float scale, bool causal,
-                       cudaStream_t stream) {
-  if (d == 64)
-    return causal ? launch_bwd<64, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream)
-                  : launch_bwd<64, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream);
-  return causal ? launch_bwd<128, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream)
-                : launch_bwd<128, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, BH, N, scale, stream);
+                       void* workspace, const Shape& s, cudaStream_t stream) {
+  const bool causal = s.mask != 0;
+  if (s.d == 64)
+    return causal ? launch_bwd<64, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream)
+                  : launch_bwd<64, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
+  return causal ? launch_bwd<128, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream)
+                : launch_bwd<128, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
+}
+
+// Argument checks of the forward (nothing is launched when one fails), then the launch.
+fa_status fwd_checked(const void* q, const void* k, const void* v, void* o, float* lse,
+                      const Shape& s, void* stream) {
+  fa_status st = check_shape(s);
+  if (st != FA_OK) return st;
+  if (!q || !k || !v || !o || !lse) return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return set_err(FA_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  const void* ins[3] = {q, k, v};
+  const size_t insz[3] = {s.q_bytes(), s.kv_bytes(), s.kv_bytes()};
+  for (int b = 0; b < 3; ++b)
+    if (overlaps(o, s.q_bytes(), ins[b], insz[b]) || overlaps(lse, s.lse_bytes(), ins[b], insz[b]))
+      return set_err(FA_ERR_INVALID_ARG, "outputs must not alias inputs");
+  if (overlaps(o, s.q_bytes(), lse, s.lse_bytes()))
+    return set_err(FA_ERR_INVALID_ARG, "o and lse overlap");
+  DeviceState* ds = device_state(&st);
+  if (!ds) return st;
+  return fwd_dispatch(ds, q, k, v, o, lse, s, static_cast<cudaStream_t>(stream));
+}
+
+size_t bwd_workspace(const Shape& s) {
+  return fa::bwd_workspace_bytes(static_cast<size_t>(s.B) * s.H, s.N_q, s.d);
+}
+
+// Argument checks of the backward (nothing is launched when one fails), then the launch.
+fa_status bwd_checked(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                      const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                      size_t workspace_bytes, const Shape& s, void* stream) {
+  fa_status st = check_shape(s);
+  if (st != FA_OK) return st;
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv)
+    return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
+  const void* ptrs[10] = {q, k, v, o, dO, lse, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return set_err(FA_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  const size_t need = bwd_workspace(s);
+  if (!workspace || workspace_bytes < need)
+    return set_err(FA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
+                   need);
+  const size_t qb = s.q_bytes(), kvb = s.kv_bytes();
+  const void* ins[6] = {q, k, v, o, dO, lse};
+  const size_t insz[6] = {qb, kvb, kvb, qb, qb, s.lse_bytes()};
+  void* outs[4] = {dq, dk, dv, workspace};
+  const size_t outsz[4] = {qb, kvb, kvb, need};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlaps(outs[a], outsz[a], ins[b], insz[b]))
+        return set_err(FA_ERR_INVALID_ARG, "outputs/workspace must not alias inputs");
+    for (int b = a + 1; b < 4; ++b)
+      if (overlaps(outs[a], outsz[a], outs[b], outsz[b]))
+        return set_err(FA_ERR_INVALID_ARG, "outputs/workspace must not overlap each other");
+  }
+  DeviceState* ds = device_state(&st);
+  if (!ds) return st;
+  return bwd_dispatch(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s,
+                      static_cast<cudaStream_t>(stream));
+}
+
+Shape from_public(const fa_attn_shape* p) {
+  return Shape{p->B, p->H, p->H_kv, p->N_q, p->N_kv, p->d, p->scale, p->mask};
 }
 
 // ---- failure-detection self-test ----
@@ -378,27 +479,14 @@ const char* fa_version(void) { return "exact_io_aware_66_b200 0.1 (sm_100a)"; }
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int N, int d, float scale, int causal, void* stream) {
   g_err[0] = '\0';
-  fa_status st = check_sizes(B, H, N, d, scale);
-  if (st != FA_OK) return st;
-  if (!q || !k || !v || !o || !lse) return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
-    return set_err(FA_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  const size_t tbytes = static_cast<size_t>(B) * H * N * d * 2;
-  const size_t lbytes = static_cast<size_t>(B) * H * N * 4;
-  const void* ins[3] = {q, k, v};
-  for (const void* in : ins)
-    if (overlaps(o, tbytes, in, tbytes) || overlaps(lse, lbytes, in, tbytes))
-      return set_err(FA_ERR_INVALID_ARG, "outputs must not alias inputs");
-  if (overlaps(o, tbytes, lse, lbytes)) return set_err(FA_ERR_INVALID_ARG, "o and lse overlap");
-  DeviceState* ds = device_state(&st);
-  if (!ds) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int BH = B * H;
-  if (d == 64)
-    return causal ? launch_fwd<64, true>(ds, q, k, v, o, lse, BH, N, scale, s)
-                  : launch_fwd<64, false>(ds, q, k, v, o, lse, BH, N, scale, s);
-  return causal ? launch_fwd<128, true>(ds, q, k, v, o, lse, BH, N, scale, s)
-                : launch_fwd<128, false>(ds, q, k, v, o, lse, BH, N, scale, s);
+  return fwd_checked(q, k, v, o, lse, Shape{B, H, H, N, N, d, scale, causal ? 1 : 0}, stream);
+}
+
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const fa_attn_shape* shape, void* stream) {
+  g_err[0] = '\0';
+  if (!shape) return set_err(FA_ERR_INVALID_ARG, "null shape");
+  return fwd_checked(q, k, v, o, lse, from_public(shape), stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -406,40 +494,31 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return fa::bwd_workspace_bytes(static_cast<size_t>(B) * H, N, d);
 }
 
+size_t fa_bwd_ex_workspace_size(const fa_attn_shape* shape) {
+  if (!shape) return 0;
+  const Shape s = from_public(shape);
+  const char saved = g_err[0];
+  const bool ok = check_shape(s) == FA_OK;
+  if (saved == '\0') g_err[0] = '\0';
+  return ok ? bwd_workspace(s) : 0;
+}
+
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                  const float* lse, void* dq, void* dk, void* dv, void* workspace,
                  size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
                  void* stream) {
   g_err[0] = '\0';
-  fa_status st = check_sizes(B, H, N, d, scale);
-  if (st != FA_OK) return st;
-  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv)
-    return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
-  const void* ptrs[10] = {q, k, v, o, dO, lse, dq, dk, dv, workspace};
-  for (const void* ptr : ptrs)
-    if (ptr && !aligned16(ptr)) return set_err(FA_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  const size_t need = fa_bwd_workspace_size(B, H, N, d);
-  if (!workspace || workspace_bytes < need)
-    return set_err(FA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
-                   need);
-  const size_t tbytes = static_cast<size_t>(B) * H * N * d * 2;
-  const size_t lbytes = static_cast<size_t>(B) * H * N * 4;
-  const void* ins[6] = {q, k, v, o, dO, lse};
-  const size_t insz[6] = {tbytes, tbytes, tbytes, tbytes, tbytes, lbytes};
-  void* outs[4] = {dq, dk, dv, workspace};
-  const size_t outsz[4] = {tbytes, tbytes, tbytes, need};
-  for (int a = 0; a < 4; ++a) {
-    for (int b = 0; b < 6; ++b)
-      if (overlaps(outs[a], outsz[a], ins[b], insz[b]))
-        return set_err(FA_ERR_INVALID_ARG, "outputs/workspace must not alias inputs");
-    for (int b = a + 1; b < 4; ++b)
-      if (overlaps(outs[a], outsz[a], outs[b], outsz[b]))
-        return set_err(FA_ERR_INVALID_ARG, "outputs/workspace must not overlap each other");
-  }
-  DeviceState* ds = device_state(&st);
-  if (!ds) return st;
-  return bwd_dispatch(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, B * H, N, d, scale,
-                      causal != 0, static_cast<cudaStream_t>(stream));
+  return bwd_checked(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes,
+                     Shape{B, H, H, N, N, d, scale, causal ? 1 : 0}, stream);
+}
+
+fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                    const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                    size_t workspace_bytes, const fa_attn_shape* shape, void* stream) {
+  g_err[0] = '\0';
+  if (!shape) return set_err(FA_ERR_INVALID_ARG, "null shape");
+  return bwd_checked(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes,
+                     from_public(shape), stream);
 }
 
 fa_status fa_profile_enable(int on) {
@@ -482,7 +561,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          const void* dO, const float* lse, void* dq, void* dk, void* dv, int B,
                          int H, int N, int d, float scale, int causal, void* stream) {
   g_err[0] = '\0';
-  fa_status st = check_sizes(B, H, N, d, scale);
+  const Shape shape{B, H, H, N, N, d, scale, causal ? 1 : 0};
+  fa_status st = check_shape(shape);
   if (st != FA_OK) return st;
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
   if (need > kNoAllocScratchBytes)
@@ -539,8 +619,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   // The first kernel of the backward rewrites every scratch byte the later ones read (dQ
   // accumulator zeroed, D and -lse*log2e recomputed), so the previous call's contents do not
   // matter.
-  st = bwd_dispatch(&local, q, k, v, o, dO, lse, dq, dk, dv, g_noalloc[dev].scratch, B * H, N, d,
-                    scale, causal != 0, static_cast<cudaStream_t>(stream));
+  st = bwd_dispatch(&local, q, k, v, o, dO, lse, dq, dk, dv, g_noalloc[dev].scratch, shape,
+                    static_cast<cudaStream_t>(stream));
   {
     std::lock_guard<std::mutex> lock(g_mu);
     std::memcpy(g_noalloc[dev].bwd_attr, local.bwd_attr, sizeof(local.bwd_attr));

@@ -151,11 +151,14 @@ struct BwdLayout {
 
 struct BwdParams {
   int* status;
-  int N;
-  int BH;
-  int n_kv;        // ceil(N / 128)
+  int N;           // query rows per head
+  int N_kv;        // key/value rows per head
+  int BH_kv;       // batch * key/value heads (one CTA row of the grid per key/value head)
+  int qgroup;      // query heads per key/value head
+  int off;         // causal offset: key j visible to query i iff j <= i + off
+  int n_kv;        // ceil(N_kv / 128)
   int n_q;         // ceil(N / 64)
-  int group;       // heads per scheduling group
+  int group;       // key/value heads per scheduling group
   float scale;
   float scale_log2;
 };
@@ -187,12 +190,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int per_group = p.group * p.n_kv;
   const int g0 = static_cast<int>(blockIdx.x / per_group) * p.group;
   const int r_in = static_cast<int>(blockIdx.x % per_group);
-  const int gcur = min(p.group, p.BH - g0);
+  const int gcur = min(p.group, p.BH_kv - g0);
   const int j = r_in / gcur;
-  const int bh = g0 + r_in % gcur;
+  const int bh = g0 + r_in % gcur;  // key/value head
   const int k0 = 128 * j;
-  const int qi0 = CAUSAL ? 2 * j : 0;  // first query tile (64 rows) that sees this key tile
-  const int n_i = p.n_q - qi0;
+  // First 64-row query tile with a query that sees a key of this tile (j <= i + off), and the
+  // iterations: every query head that shares this key/value head, times its query tiles.
+  const int qi0 = CAUSAL ? max(0, k0 - p.off) / 64 : 0;
+  const int n_qt = max(0, p.n_q - qi0);
+  const int n_i = p.qgroup * n_qt;
+  auto q_head = [&](int it) { return bh * p.qgroup + it / n_qt; };
+  auto q_tile = [&](int it) { return qi0 + it % n_qt; };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -238,7 +246,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (int i = 0; i < n_i && ok; ++i) {
       const int b = i & 1, st = i % QS;
-      const int qi = qi0 + i;
+      const int qi = q_tile(i);
       ok = warp_wait(bar(L::bQFull + st), (i / QS) & 1, abort_flag) &&
            warp_wait(bar(L::bSdPFull + b), (i >> 1) & 1, abort_flag) &&
            (i < 2 || warp_wait(bar(L::bDSFree + b), ((i >> 1) & 1) ^ 1, abort_flag));
@@ -253,7 +261,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* lse2 = reinterpret_cast<const float*>(gbase + L::kRow + st * 512) + 32 * w;
       const float* Dv = reinterpret_cast<const float*>(gbase + L::kRow + st * 512 + 256) + 32 * w;
       const int qbase = 64 * qi + 32 * w;
-      const bool need_mask = (CAUSAL && qi <= 2 * j + 1) || (qbase + 32 > p.N) || (k0 + 128 > p.N);
+      const bool need_mask = (CAUSAL && qbase + p.off < k0 + 127) || (qbase + 32 > p.N) ||
+                             (k0 + 128 > p.N_kv);
       uint32_t pk[16], dsk[16];
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
 #pragma unroll
@@ -275,7 +284,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int q = qbase + c + e;
-            if (q >= p.N || key >= p.N || (CAUSAL && q < key)) {
+            if (q >= p.N || key >= p.N_kv || (CAUSAL && q + p.off < key)) {
               pr[e] = 0.f;
               dsr[e] = 0.f;
             }
@@ -299,7 +308,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     if (!ok) fail(p.status, abort_flag, 5);
     // ------------------------------------------------------------ dV / dK epilogue -------
-    if (ok && warp_wait(bar(L::bAccDone), 0, abort_flag)) {
+    if (ok && (n_i == 0 || warp_wait(bar(L::bAccDone), 0, abort_flag))) {
       tc_fence_after();
       // warpgroup 0 stores dV (stage-0 Q/dO space), warpgroup 1 stores dK * scale (stage 1)
       const uint32_t tcol = w == 0 ? L::tDV : L::tDK;
@@ -309,9 +318,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + tcol + c + lane_off, v);
-        tmem_ld_wait();
-        reg_fence(v);
+        if (n_i > 0) {
+          tmem_ld_32x32b_x32(tmem + tcol + c + lane_off, v);
+          tmem_ld_wait();
+          reg_fence(v);
+        } else {  // no query sees these keys: dK = dV = 0 (TMEM was never written)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint4 u;
@@ -364,7 +378,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_reduce_add_3d(&tmDQacc, stage_s, 32 * wq, 64 * (qi0 + i), bh);
+        tma_reduce_add_3d(&tmDQacc, stage_s, 32 * wq, 64 * q_tile(i), q_head(i));
         bulk_commit_group();
       }
     }
@@ -434,7 +448,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         umma_commit(bar(L::bQEmpty + st));
         umma_commit(bar(L::bDSFree + b));
       };
-      bool ok = mbar_wait(bar(L::bKV), 0, abort_flag);
+      bool ok = n_i == 0 || mbar_wait(bar(L::bKV), 0, abort_flag);
       for (int i = 0; i < n_i && ok; ++i) {
         const int b = i & 1, st = i % QS;
         ok = mbar_wait(bar(L::bQFull + st), (i / QS) & 1, abort_flag) &&
@@ -449,7 +463,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           second_half(i - 1);
         }
       }
-      if (ok) {
+      if (ok && n_i > 0) {
         const int i = n_i - 1;
         ok = mbar_wait(bar(L::bEwDone + (i & 1)), (i >> 1) & 1, abort_flag);
         if (ok) {
@@ -468,11 +482,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == 13) {
     // --------------------------------------------------------------------- TMA ----------
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(L::bKV), 2 * L::kKVTile);
+      if (n_i > 0) {
+        mbar_arrive_expect_tx(bar(L::bKV), 2 * L::kKVTile);
 #pragma unroll
-      for (int bx = 0; bx < L::kBoxes; ++bx) {
-        tma_load_3d(sbase + L::kK + bx * L::kKVBox, &tmK, bar(L::bKV), 64 * bx, k0, bh);
-        tma_load_3d(sbase + L::kV + bx * L::kKVBox, &tmV, bar(L::bKV), 64 * bx, k0, bh);
+        for (int bx = 0; bx < L::kBoxes; ++bx) {
+          tma_load_3d(sbase + L::kK + bx * L::kKVBox, &tmK, bar(L::bKV), 64 * bx, k0, bh);
+          tma_load_3d(sbase + L::kV + bx * L::kKVBox, &tmV, bar(L::bKV), 64 * bx, k0, bh);
+        }
       }
       int issued = 0;
       for (int i = 0; i < n_i; ++i) {
@@ -481,24 +497,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           fail(p.status, abort_flag, 5);
           break;
         }
-        const int q0 = 64 * (qi0 + i);
+        const int q0 = 64 * q_tile(i), qh = q_head(i);
         mbar_arrive_expect_tx(bar(L::bQFull + st), 2 * L::kQTile + 512);
 #pragma unroll
         for (int bx = 0; bx < L::kBoxes; ++bx) {
           tma_load_3d(sbase + L::kQ + st * 2 * L::kQTile + bx * L::kQBox, &tmQ,
-                      bar(L::bQFull + st), 64 * bx, q0, bh);
+                      bar(L::bQFull + st), 64 * bx, q0, qh);
           tma_load_3d(sbase + L::kDO + st * 2 * L::kQTile + bx * L::kQBox, &tmDO,
-                      bar(L::bQFull + st), 64 * bx, q0, bh);
+                      bar(L::bQFull + st), 64 * bx, q0, qh);
         }
-        tma_load_3d(sbase + L::kRow + st * 512, &tmLse2, bar(L::bQFull + st), q0, bh, 0);
-        tma_load_3d(sbase + L::kRow + st * 512 + 256, &tmD, bar(L::bQFull + st), q0, bh, 0);
+        tma_load_3d(sbase + L::kRow + st * 512, &tmLse2, bar(L::bQFull + st), q0, qh, 0);
+        tma_load_3d(sbase + L::kRow + st * 512 + 256, &tmD, bar(L::bQFull + st), q0, qh, 0);
         issued = i + 1;
       }
       if (*abort_flag) {
         volatile int never = 0;
         for (int i = max(0, issued - QS); i < issued; ++i)
           mbar_wait(bar(L::bQFull + (i % QS)), (i / QS) & 1, &never);
-        mbar_wait(bar(L::bKV), 0, &never);
+        if (n_i > 0) mbar_wait(bar(L::bKV), 0, &never);
       }
     }
   }

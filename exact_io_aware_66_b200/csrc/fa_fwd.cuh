@@ -65,8 +65,11 @@ struct FwdLayout {
 struct FwdParams {
   float* lse;       // [BH, N] fp32
   int* status;      // device status word (FA_ERR_TIMEOUT on a timed-out wait)
-  int N;            // sequence length
-  int BH;           // batch * heads
+  int N;            // query rows per head
+  int N_kv;         // key/value rows per head
+  int BH;           // batch * query heads
+  int group;        // query heads per key/value head (1 unless K/V heads are shared)
+  int off;          // causal offset: key j visible to query i iff j <= i + off
   int n_qblocks;    // ceil(N / 256)
   float scale;      // softmax scale
   float scale_log2; // scale * log2(e)
@@ -126,11 +129,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // the block index) are scheduled first.
   const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x / p.BH);
   const int bh = static_cast<int>(blockIdx.x % p.BH);
+  const int bh_kv = bh / p.group;  // key/value head of this query head
   const int q0 = qb * 256;
-  const int nkv = (p.N + 127) / 128;
+  const int nkv = (p.N_kv + 127) / 128;
+  // Key tiles each query tile visits: all of them, or (causal) up to the one holding the last
+  // key its last row sees; 0 when no row of the tile sees any key.
   int n_t[2];
 #pragma unroll
-  for (int t = 0; t < 2; ++t) n_t[t] = CAUSAL ? min(nkv, 2 * qb + t + 1) : nkv;
+  for (int t = 0; t < 2; ++t) {
+    const int last_key = q0 + 128 * t + 127 + p.off;
+    n_t[t] = !CAUSAL ? nkv : (last_key < 0 ? 0 : min(nkv, last_key / 128 + 1));
+  }
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -170,7 +179,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int row = threadIdx.x & 127;
     const uint32_t tS = tmem + t * 128 + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int q_row = q0 + t * 128 + row;
-    const int tile_idx = 2 * qb + t;
     const float sl2 = p.scale_log2;
     float m = -INFINITY;
     float l = 0.f;   // sum of the fp32 exponentials: gives lse
@@ -190,9 +198,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tmem_ld_wait();
       reg_fence(s);
       const int kv0 = j * 128;
-      const bool need_mask = (CAUSAL && j == tile_idx) || (kv0 + 128 > p.N);
+      const bool need_mask = (CAUSAL && kv0 + 127 > q0 + t * 128 + p.off) || (kv0 + 128 > p.N_kv);
       if (need_mask) {
-        const int lim = CAUSAL ? min(q_row + 1, p.N) : p.N;  // keys [0, lim) visible
+        const int lim = CAUSAL ? min(q_row + 1 + p.off, p.N_kv) : p.N_kv;  // keys [0, lim)
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
@@ -215,7 +223,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         alpha = ex2_approx((m - m_tile) * sl2);  // 0 on the first tile
         m = m_tile;
       }
-      const float nb = -m * sl2;
+      // a row that has seen no key yet keeps m = -inf; its exponentials are then exactly 0
+      const float nb = m == -INFINITY ? 0.f : -m * sl2;
       const uint64_t sl2x2 = f2_pack(sl2, sl2), nbx2 = f2_pack(nb, nb);
       uint64_t lsum[4] = {0, 0, 0, 0}, rsum[4] = {0, 0, 0, 0};  // (0.f, 0.f) pairs
       uint32_t pk[64];
@@ -267,8 +276,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     s_rowl[t * 128 + row] = lr;
     mbar_arrive(bar(L::bFinal + t));
+    // rows that saw no key: O = 0 and lse = -inf
     if (!*abort_flag && q_row < p.N)
-      p.lse[static_cast<size_t>(bh) * p.N + q_row] = (m * sl2 + lg2_approx(l)) * 0.69314718055994531f;
+      p.lse[static_cast<size_t>(bh) * p.N + q_row] =
+          l > 0.f ? (m * sl2 + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
   } else if (warp < 12) {
     // ----------------------------------------------------------------- epilogue ----------
     setmaxnreg_dec<kFwdRegEpilogue>();
@@ -278,22 +289,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // Epilogue: O = O_acc / l  ->  bf16  ->  swizzled staging (reusing the Q tile)  ->  TMA.
     // Each warp stores its own 32 rows (box 64 x 32), so no cross-warp barrier is needed.
     for (int t = 0; t < 2 && ok; ++t) {
+      // A tile that saw no key has no MMA ordering its staging writes after the Q load into
+      // the same shared memory, so it waits for that load itself.
       if (!warp_wait(bar(L::bFinal + t), 0, abort_flag) ||
-          !warp_wait(bar(L::bODone + t), (n_t[t] - 1) & 1, abort_flag)) {
+          (n_t[t] > 0 && !warp_wait(bar(L::bODone + t), (n_t[t] - 1) & 1, abort_flag)) ||
+          (n_t[t] == 0 && !warp_wait(bar(L::bQ), 0, abort_flag))) {
         fail(p.status, abort_flag, 5);
         ok = false;
         break;
       }
       tc_fence_after();
-      const float inv_l = 1.0f / s_rowl[t * 128 + row];
+      const float lr_row = s_rowl[t * 128 + row];
+      const float inv_l = lr_row > 0.f ? 1.0f / lr_row : 0.f;
+      const bool empty_tile = n_t[t] == 0;  // no PV ever wrote this O accumulator
       const uint32_t tO = tmem + 256 + t * D + lane_off;
       uint8_t* stage = gbase + L::kQ + t * L::kTileBytes;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
-        tmem_ld_32x32b_x32(tO + c, o);
-        tmem_ld_wait();
-        reg_fence(o);
+        if (!empty_tile) {
+          tmem_ld_32x32b_x32(tO + c, o);
+          tmem_ld_wait();
+          reg_fence(o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {  // four 16-byte chunks of 8 columns
           uint4 v;
@@ -351,10 +372,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           umma_ts(d, a + kk * 8, sdesc_advance(b0, kk * 2048), idesc_pv, 1u);
         umma_commit(bar(L::bODone + t));
       };
-      bool ok = mbar_wait(bar(L::bQ), 0, abort_flag) && wait_full(0);
-      if (ok) {
+      bool ok = n_t[1] == 0 || (mbar_wait(bar(L::bQ), 0, abort_flag) && wait_full(0));
+      if (ok && n_t[1] > 0) {
         tc_fence_after();
-        issue_s(0, 0);
+        if (n_t[0] > 0) issue_s(0, 0);
         issue_s(1, 0);
         umma_commit(bar(L::bKvEmpty + 0 % ST));
       }
@@ -415,7 +436,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int b = 0; b < L::kBoxes; ++b)
             tma_load_3d(dst + b * L::kBoxBytes, w ? &tmV : &tmK, bar(L::bKvFull + st), 64 * b,
-                        128 * j, bh);
+                        128 * j, bh_kv);
           issued = tt + 1;
         }
         if (!ok) {

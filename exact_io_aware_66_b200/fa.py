@@ -38,7 +38,34 @@ SIGNATURES = {
     "fa_kernel_name": (ctypes.c_char_p, [_I]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_selftest_timeout": (_I, [_I, _P]),
+    "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P]),
+    "fa_bwd_ex_workspace_size": (_Z, [_P]),
+    "fa_bwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
 }
+
+# fa_mask values
+MASK_NONE, MASK_CAUSAL, MASK_CAUSAL_BOTTOM_RIGHT = 0, 1, 2
+
+
+class FaAttnShape(ctypes.Structure):
+    """struct fa_attn_shape of include/fa.h."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int),
+                ("N_q", ctypes.c_int), ("N_kv", ctypes.c_int), ("d", ctypes.c_int),
+                ("scale", ctypes.c_float), ("mask", ctypes.c_int)]
+
+
+def mask_code(causal) -> int:
+    """False / "none" -> no mask; True / "top_left" -> causal aligned at the top left;
+    "bottom_right" -> causal aligned at the bottom right (key j visible to query i iff
+    j <= i + N_kv - N_q)."""
+    if causal is False or causal is None or causal == "none":
+        return MASK_NONE
+    if causal is True or causal == "top_left":
+        return MASK_CAUSAL
+    if causal == "bottom_right":
+        return MASK_CAUSAL_BOTTOM_RIGHT
+    raise ValueError(f"unknown mask {causal!r}")
+
 
 KERNEL_KINDS = 4
 
@@ -188,22 +215,77 @@ def fa_check_status(stream=None):
     _check("fa_check_status", lib().fa_check_status(_stream_handle(stream)))
 
 
-def attention_forward(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
-    """Returns (o, lse) for bf16 CUDA tensors q, k, v of shape [B, H, N, d]."""
+def _shape(q, k, v, causal, scale) -> FaAttnShape:
+    B, H, N_q, d = _dims(q)
+    Bk, H_kv, N_kv, dk = _dims(k)
+    if Bk != B or dk != d:
+        raise ValueError("k must be [B, H_kv, N_kv, d] with q's B and d")
+    if _dims(v) != (B, H_kv, N_kv, d):
+        raise ValueError("v shape mismatch")
+    scale = default_scale(d) if scale is None else float(scale)
+    return FaAttnShape(B, H, H_kv, N_q, N_kv, d, scale, mask_code(causal))
+
+
+def fa_fwd_ex(q, k, v, o, lse, causal=False, scale: float | None = None, stream=None):
+    """Forward for q [B,H,N_q,d] and k, v [B,H_kv,N_kv,d] (H a multiple of H_kv) into
+    caller-allocated o (like q) and lse (fp32 [B,H,N_q]); causal as in mask_code."""
+    s = _shape(q, k, v, causal, scale)
+    if _dims(o) != (s.B, s.H, s.N_q, s.d):
+        raise ValueError("o shape mismatch")
+    if tuple(lse.shape) != (s.B, s.H, s.N_q):
+        raise ValueError("lse must be [B, H, N_q]")
+    ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(lse, "lse", torch.float32)]
+    _check("fa_fwd_ex", lib().fa_fwd_ex(*ptrs, ctypes.byref(s), _stream_handle(stream)))
+
+
+def fa_bwd_ex_workspace_size(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int,
+                             causal=False) -> int:
+    s = FaAttnShape(B, H, H_kv, N_q, N_kv, d, default_scale(d) if d > 0 else 1.0,
+                    mask_code(causal))
+    return int(lib().fa_bwd_ex_workspace_size(ctypes.byref(s)))
+
+
+def fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, causal=False,
+              scale: float | None = None, stream=None):
+    """Backward for the shapes of fa_fwd_ex into caller-allocated dq (like q), dk, dv (like k)
+    with a caller-owned workspace of at least fa_bwd_ex_workspace_size bytes."""
+    s = _shape(q, k, v, causal, scale)
+    for t, n in ((o, "o"), (do, "do"), (dq, "dq")):
+        if _dims(t) != (s.B, s.H, s.N_q, s.d):
+            raise ValueError(f"{n} shape mismatch")
+    for t, n in ((dk, "dk"), (dv, "dv")):
+        if _dims(t) != (s.B, s.H_kv, s.N_kv, s.d):
+            raise ValueError(f"{n} shape mismatch")
+    if tuple(lse.shape) != (s.B, s.H, s.N_q):
+        raise ValueError("lse must be [B, H, N_q]")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(do, "do"),
+            _req(lse, "lse", torch.float32), _req(dq, "dq"), _req(dk, "dk"), _req(dv, "dv")]
+    wbytes = workspace.numel() * workspace.element_size()
+    _check("fa_bwd_ex", lib().fa_bwd_ex(*ptrs, workspace.data_ptr(), wbytes, ctypes.byref(s),
+                                        _stream_handle(stream)))
+
+
+def attention_forward(q, k, v, causal=False, scale: float | None = None, stream=None):
+    """Returns (o, lse) for bf16 CUDA tensors q [B, H, N_q, d] and k, v [B, H_kv, N_kv, d]
+    (H_kv = H and N_kv = N_q in the square case); causal as in mask_code."""
     B, H, N, d = _dims(q)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    fa_fwd(q, k, v, o, lse, causal, scale, stream)
+    fa_fwd_ex(q, k, v, o, lse, causal, scale, stream)
     return o, lse
 
 
-def attention_backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
+def attention_backward(q, k, v, o, do, lse, causal=False, scale: float | None = None,
                        stream=None, workspace=None):
-    """Returns (dq, dk, dv). Allocates the workspace unless one is given."""
+    """Returns (dq, dk, dv) for the shapes of attention_forward. Allocates the workspace
+    unless one is given."""
     B, H, N, d = _dims(q)
+    _, H_kv, N_kv, _ = _dims(k)
     if workspace is None:
-        workspace = torch.empty(fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8,
-                                device=q.device)
+        workspace = torch.empty(fa_bwd_ex_workspace_size(B, H, H_kv, N, N_kv, d, causal),
+                                dtype=torch.uint8, device=q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, causal, scale, stream)
+    fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, causal, scale, stream)
     return dq, dk, dv

@@ -85,6 +85,18 @@ def make_inputs(B: int, H: int, N: int, d: int, seed: int, mult: float = 1.0,
     return out
 
 
+def make_inputs_ex(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int, seed: int) -> dict:
+    """{'q','do'} of shape [B, H, N_q, d] and {'k','v'} of shape [B, H_kv, N_kv, d], contiguous
+    bf16 CPU tensors of standard normal draws (for grouped heads and unequal lengths)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    out = {}
+    for name, (h, n) in (("q", (H, N_q)), ("k", (H_kv, N_kv)), ("v", (H_kv, N_kv)),
+                         ("do", (H, N_q))):
+        out[name] = torch.randn(B, h, n, d, dtype=torch.float32, generator=g).to(
+            torch.bfloat16).contiguous()
+    return out
+
+
 def workload_inputs(w: Workload, with_do: bool | None = None) -> dict:
     if with_do is None:
         with_do = w.backward

@@ -53,6 +53,40 @@ typedef enum {
 
 /* Limits: d in {64, 128}; B, H, N >= 1; B*H*N < 2^31; B*H*ceil(N/256) < 2^31. */
 
+/* Masks of the extended entry points. */
+typedef enum {
+  FA_MASK_NONE = 0,                /* every key visible to every query */
+  FA_MASK_CAUSAL = 1,              /* key j visible to query i iff j <= i (top-left aligned) */
+  FA_MASK_CAUSAL_BOTTOM_RIGHT = 2  /* iff j <= i + N_kv - N_q: the last query sees every key,
+                                      as when new queries attend to a longer cached context */
+} fa_mask;
+
+/* Shape of the extended entry points: q, o, dO, dq are bf16 [B, H, N_q, d]; k, v, dk, dv are
+ * bf16 [B, H_kv, N_kv, d]; lse is fp32 [B, H, N_q]. H must be a multiple of H_kv: query head h
+ * uses key/value head h / (H / H_kv) (grouped heads; H_kv = 1 is a single shared K/V head),
+ * and dk, dv of a key/value head sum over the query heads that share it. A query row that sees
+ * no key (FA_MASK_CAUSAL_BOTTOM_RIGHT with N_q > N_kv) gets o = 0, lse = -inf and dq = 0.
+ * Limits: d in {64, 128}; all sizes >= 1; B*H*N_q and B*H_kv*N_kv < 2^31. */
+typedef struct {
+  int B, H, H_kv, N_q, N_kv, d;
+  float scale; /* finite, > 0; normally 1/sqrt(d) */
+  int mask;    /* an fa_mask value */
+} fa_attn_shape;
+
+/* Forward for an fa_attn_shape (fa_fwd is the case H_kv = H, N_q = N_kv = N). The pages define
+ * the square, equal-head case; these shapes apply the same definition with the mask above. */
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const fa_attn_shape* shape, void* stream);
+
+/* Workspace bytes fa_bwd_ex needs (fp32 dQ accumulator and row terms for B*H*N_q rows); 0 for an
+ * invalid shape. */
+size_t fa_bwd_ex_workspace_size(const fa_attn_shape* shape);
+
+/* Backward for an fa_attn_shape; arguments as fa_bwd. */
+fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                    const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                    size_t workspace_bytes, const fa_attn_shape* shape, void* stream);
+
 /* Forward. Writes o (bf16 [B,H,N,d]) and lse (fp32 [B,H,N]).
  * scale: the softmax scale (finite, > 0), normally 1/sqrt(d). causal: 0 or 1.
  * stream: a cudaStream_t passed as void*. */

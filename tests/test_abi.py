@@ -117,3 +117,40 @@ def test_no_cpu_fallback_in_product_package():
 def test_selftest_timeout_rejects_bad_limit_without_gpu(lib):
     assert lib.fa_selftest_timeout(0, None) == 1
     assert lib.fa_selftest_timeout(10 ** 8, None) == 1
+
+
+def _fwd_ex_raw(lib, B=1, H=2, H_kv=1, N_q=100, N_kv=300, d=64, scale=0.125, mask=2, o=1 << 20,
+                lse=2 << 20):
+    s = fa.FaAttnShape(B, H, H_kv, N_q, N_kv, d, scale, mask)
+    return lib.fa_fwd_ex(16, 1 << 16, 2 << 16, o, lse, ctypes.byref(s), None)
+
+
+def test_fwd_ex_validation_without_gpu(lib):
+    assert lib.fa_fwd_ex(16, 32, 48, 1 << 20, 2 << 20, None, None) == 1  # null shape
+    assert _fwd_ex_raw(lib, H=3, H_kv=2) == 1  # H not a multiple of H_kv
+    assert "multiple" in fa.fa_last_error_string()
+    assert _fwd_ex_raw(lib, mask=3) == 1
+    assert _fwd_ex_raw(lib, N_kv=0) == 1
+    assert _fwd_ex_raw(lib, d=80) == 2
+    # o (B*H*N_q*d*2 = 25600 bytes from 1<<16 - 25600 + 16) would overlap k at 1<<16
+    assert _fwd_ex_raw(lib, o=(1 << 16) - 1024) == 1
+    # k and v are B*H_kv*N_kv*d*2 = 38400 bytes: an lse placed inside v overlaps it
+    assert _fwd_ex_raw(lib, lse=(2 << 16) + 1024) == 1
+
+
+def test_bwd_ex_workspace_size(lib):
+    s = fa.FaAttnShape(2, 4, 2, 100, 300, 64, 0.125, 1)
+    ws = lib.fa_bwd_ex_workspace_size(ctypes.byref(s))
+    # the workspace scales with the query rows B*H*N_q, not with the keys
+    assert ws == fa.fa_bwd_workspace_size(2, 4, 100, 64)
+    assert fa.fa_bwd_ex_workspace_size(2, 4, 2, 100, 300, 64, True) == ws
+    assert fa.fa_bwd_ex_workspace_size(2, 4, 3, 100, 300, 64, True) == 0
+    assert lib.fa_bwd_ex_workspace_size(None) == 0
+
+
+def test_mask_code():
+    assert fa.mask_code(False) == 0 and fa.mask_code("none") == 0
+    assert fa.mask_code(True) == 1 and fa.mask_code("top_left") == 1
+    assert fa.mask_code("bottom_right") == 2
+    with pytest.raises(ValueError):
+        fa.mask_code("diagonal")
