@@ -21,3 +21,4 @@ from .attention import (  # noqa: F401
     online_softmax_stats,
     tiled_attention_forward,
 )
+from .dropout import dropout_keep, dropout_p8, keep_scale, philox4x32_10  # noqa: F401

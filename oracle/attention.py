@@ -34,6 +34,13 @@ What is computed, and where it is defined:
       D_i = sum_c dO_ic O_ic          (= sum_j P_ij dP_ij, the softmax-Jacobian row term)
       dS = P o (dP - D)               (o = elementwise product; masked entries are exactly 0)
       dQ = scale * dS K,   dK = scale * dS^T Q
+* Dropout (optional, ``dropout=(p, seed, offset)``): inverted dropout on P, applied where
+  "How FlashAttention Actually Works", section "The GPU Memory Wall: HBM vs. SRAM", places it
+  (on the softmax matrix, before the product with V). With Z the keep decisions of
+  ``oracle.dropout`` and r = 256 / (256 - p8) the keep scale:
+      O_i = r sum_j Z_ij P_ij v_j,   lse_i unchanged (the undropped softmax)
+      dV = r (Z o P)^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,  dS = P o (r Z o dP - D)
+  (D is still rowsum(dO o O) with the dropped O: sum_j P_ij r Z_ij dP_ij = dO_i . O_i).
 * Tiled forward with online softmax. "How does FlashAttention optimize memory and speed via
   tiling?" (iloveeagents.com), section "Core Technical Innovations", item 2 gives the update
       m^(2) = max(m^(1), m~),  d^(2) = e^{m^(1) - m^(2)} d^(1) + e^{m~ - m^(2)} d~
@@ -53,6 +60,8 @@ this).
 from __future__ import annotations
 
 import numpy as np
+
+from .dropout import dropout_keep, dropout_p8, keep_scale
 
 __all__ = [
     "attention_probabilities",
@@ -118,10 +127,27 @@ def _softmax_block(s: np.ndarray, mask: np.ndarray | None):
     return m, e, e.sum(axis=1)
 
 
-def _finish(e, l, m, v):
-    """O = e V / l and lse = m + ln l, with O = 0 and lse = -inf for rows that see no key."""
+def _dropout(dropout):
+    """(p8, keep scale, seed, offset) for ``dropout=(p, seed, offset)``, or None."""
+    if dropout is None:
+        return None
+    p, seed, offset = dropout
+    p8 = dropout_p8(p)
+    return p8, keep_scale(p8), int(seed), int(offset)
+
+
+def _flat_head(idx, q_shape) -> int:
+    """Flattened query-head index (b * H + h for [B, H, N, d]) of leading index `idx`."""
+    lead = q_shape[:-2]
+    return int(np.ravel_multi_index(idx, lead)) if lead else 0
+
+
+def _finish(e, l, m, v, z=None, r=1.0):
+    """O = e V / l and lse = m + ln l, with O = 0 and lse = -inf for rows that see no key.
+    With dropout keep decisions z and keep scale r: O = r (z o e) V / l."""
     empty = l == 0.0
-    o = (e @ v) / np.where(empty, 1.0, l)[:, None]
+    num = (e @ v) if z is None else r * ((e * z) @ v)
+    o = num / np.where(empty, 1.0, l)[:, None]
     with np.errstate(divide="ignore"):
         lse = np.where(empty, -np.inf, m + np.log(np.where(empty, 1.0, l)))
     return o, lse
@@ -153,16 +179,19 @@ def attention_probabilities(q, k, scale: float, causal=False) -> np.ndarray:
     return out
 
 
-def attention_forward(q, k, v, scale: float, causal=False, block_rows: int = 512):
+def attention_forward(q, k, v, scale: float, causal=False, block_rows: int = 512,
+                      dropout=None):
     """Exact attention forward: returns (O [..., N_q, d], lse [..., N_q]) in float64.
 
     Definition: codethepapers.com, "The Problem: The Memory Wall" (P = softmax(QK^T/sqrt d),
     output P V) with the running max m and sum l of hot.atechcom.net, "The Secret Weapon:
     Online Softmax"; lse = m + ln l. Masked entries contribute exactly 0; `causal` is a mask
-    mode (see the module docstring); K/V may have fewer heads than Q (grouped heads).
+    mode (see the module docstring); K/V may have fewer heads than Q (grouped heads);
+    `dropout` = (p, seed, offset) applies inverted dropout to P (module docstring).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     mode = _mode(causal)
+    drop = _dropout(dropout)
     scale = float(np.float64(scale))
     n, nk = q.shape[-2], k.shape[-2]
     o = np.zeros(q.shape[:-1] + (v.shape[-1],), dtype=np.float64)
@@ -177,12 +206,16 @@ def attention_forward(q, k, v, scale: float, causal=False, block_rows: int = 512
             s = scale * (qh[r0:r1] @ kh[:kv_end].T)
             m, e, l = _softmax_block(s, _mask(r0, r1, n, nk, mode)[:, :kv_end]
                                      if mode != "none" else None)
-            o[idx][r0:r1], lse[idx][r0:r1] = _finish(e, l, m, vh[:kv_end])
+            z, r = None, 1.0
+            if drop is not None:
+                p8, r, seed, offset = drop
+                z = dropout_keep(_flat_head(idx, q.shape), range(r0, r1), kv_end, p8, seed, offset)
+            o[idx][r0:r1], lse[idx][r0:r1] = _finish(e, l, m, vh[:kv_end], z, r)
     return o, lse
 
 
 def attention_backward(q, k, v, do, scale: float, causal: bool = False, block_rows: int = 512,
-                       return_forward: bool = False):
+                       return_forward: bool = False, dropout=None):
     """Gradient of exact attention: returns (dQ, dK, dV) in float64 (and (O, lse) if asked).
 
     Recomputes O and lse from the definition (attention_forward), then
@@ -190,11 +223,14 @@ def attention_backward(q, k, v, do, scale: float, causal: bool = False, block_ro
     dQ = scale dS K, dK = scale dS^T Q. These are the calculus of the forward definition; the
     pages only state that scores are recomputed on chip in the backward ("How FlashAttention
     Actually Works", "The Backward Pass: Recomputation"). D uses the oracle's own fp64 O.
+    With `dropout`, the module docstring's dropout formulas apply (same keep decisions as the
+    forward).
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     mode = _mode(causal)
     scale = float(np.float64(scale))
-    o, lse = attention_forward(q, k, v, scale, mode, block_rows)
+    drop = _dropout(dropout)
+    o, lse = attention_forward(q, k, v, scale, mode, block_rows, dropout)
     n, nk = q.shape[-2], k.shape[-2]
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
@@ -214,9 +250,15 @@ def attention_backward(q, k, v, do, scale: float, causal: bool = False, block_ro
                 p = np.exp(s - lse[idx][r0:r1, None])
             if mask is not None:
                 p = np.where(mask[:, :kv_end], p, 0.0)
-            dv[kvi][:kv_end] += p.T @ doh[r0:r1]
             dp = doh[r0:r1] @ vh[:kv_end].T
-            ds = p * (dp - dd[r0:r1, None])
+            if drop is None:
+                dv[kvi][:kv_end] += p.T @ doh[r0:r1]
+                ds = p * (dp - dd[r0:r1, None])
+            else:
+                p8, r, seed, offset = drop
+                z = dropout_keep(_flat_head(idx, q.shape), range(r0, r1), kv_end, p8, seed, offset)
+                dv[kvi][:kv_end] += r * ((z * p).T @ doh[r0:r1])
+                ds = p * (r * z * dp - dd[r0:r1, None])
             dq[idx][r0:r1] = scale * (ds @ kh[:kv_end])
             dk[kvi][:kv_end] += scale * (ds.T @ qh[r0:r1])
     if return_forward:
@@ -224,7 +266,7 @@ def attention_backward(q, k, v, do, scale: float, causal: bool = False, block_ro
     return dq, dk, dv
 
 
-def attention_rows(q, k, v, scale: float, causal: bool, rows, do=None):
+def attention_rows(q, k, v, scale: float, causal: bool, rows, do=None, dropout=None):
     """Forward (and dQ) for selected query rows only; cost O(N d) per row.
 
     rows: iterable of index tuples (leading indices..., i), e.g. (b, h, i) for [B, H, N, d].
@@ -234,6 +276,7 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, do=None):
     q, k, v = _f64(q), _f64(k), _f64(v)
     do = None if do is None else _f64(do)
     mode = _mode(causal)
+    drop = _dropout(dropout)
     scale = float(np.float64(scale))
     rows = [tuple(int(t) for t in r) for r in rows]
     n, nk = q.shape[-2], k.shape[-2]
@@ -252,21 +295,26 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, do=None):
         m = s.max()
         e = np.exp(s - m)
         l = e.sum()
-        o_i = (e @ vh) / l
+        zr = 1.0  # keep decision times keep scale, per key
+        if drop is not None:
+            p8, r, seed, offset = drop
+            zr = r * dropout_keep(_flat_head(head, q.shape), [i], vis, p8, seed, offset)[0]
+        o_i = ((e * zr) @ vh) / l
         o_out[t] = o_i
         lse_out[t] = m + np.log(l)
         if do is not None:
             p = e / l
             do_i = do[head][i]
             dp = vh @ do_i
-            ds = p * (dp - do_i @ o_i)
+            ds = p * (zr * dp - do_i @ o_i)
             dq_out[t] = scale * (ds @ kh)
     if do is not None:
         return o_out, lse_out, dq_out
     return o_out, lse_out
 
 
-def attention_keys(q, k, v, do, scale: float, causal, head, keys, block_rows: int = 512):
+def attention_keys(q, k, v, do, scale: float, causal, head, keys, block_rows: int = 512,
+                   dropout=None):
     """dK and dV rows for selected keys j of one key/value head (leading index tuple `head`,
     e.g. (b, h_kv)).
 
@@ -277,6 +325,7 @@ def attention_keys(q, k, v, do, scale: float, causal, head, keys, block_rows: in
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     mode = _mode(causal)
     scale = float(np.float64(scale))
+    drop = _dropout(dropout)
     head = tuple(int(t) for t in head)
     kh, vh = k[head], v[head]
     n, nk = q.shape[-2], k.shape[-2]
@@ -290,7 +339,8 @@ def attention_keys(q, k, v, do, scale: float, causal, head, keys, block_rows: in
     dv_out = np.zeros((len(keys), vh.shape[1]))
     for qh_idx in q_heads:
         qh, doh = q[qh_idx], do[qh_idx]
-        o, lse = attention_forward(qh, kh, vh, scale, mode, block_rows)
+        bh = _flat_head(qh_idx, q.shape)
+        o, lse = _forward_one_head(qh, kh, vh, scale, mode, block_rows, bh, drop)
         dd = np.sum(doh * o, axis=1)
         for t, j in enumerate(int(x) for x in keys):
             i0 = 0 if mode == "none" else max(0, j - off)  # rows i with j <= i + off see key j
@@ -298,11 +348,35 @@ def attention_keys(q, k, v, do, scale: float, causal, head, keys, block_rows: in
                 continue
             s = scale * (qh[i0:n] @ kh[j])
             p = np.exp(s - lse[i0:n])
-            dv_out[t] += p @ doh[i0:n]
+            zr = 1.0
+            if drop is not None:
+                p8, r, seed, offset = drop
+                zr = r * dropout_keep(bh, range(i0, n), [j], p8, seed, offset)[:, 0]
+            dv_out[t] += (zr * p) @ doh[i0:n]
             dp = doh[i0:n] @ vh[j]
-            ds = p * (dp - dd[i0:n])
+            ds = p * (zr * dp - dd[i0:n])
             dk_out[t] += scale * (ds @ qh[i0:n])
     return dk_out, dv_out
+
+
+def _forward_one_head(qh, kh, vh, scale, mode, block_rows, bh, drop):
+    """attention_forward of one [N, d] head whose flattened query-head index is bh (the index
+    that selects its dropout draws)."""
+    n, nk = qh.shape[0], kh.shape[0]
+    o = np.zeros((n, vh.shape[1]))
+    lse = np.zeros(n)
+    for r0 in range(0, n, block_rows):
+        r1 = min(n, r0 + block_rows)
+        kv_end = _visible(r1 - 1, n, nk, mode)
+        s = scale * (qh[r0:r1] @ kh[:kv_end].T)
+        m, e, l = _softmax_block(s, _mask(r0, r1, n, nk, mode)[:, :kv_end]
+                                 if mode != "none" else None)
+        z, r = None, 1.0
+        if drop is not None:
+            p8, r, seed, offset = drop
+            z = dropout_keep(bh, range(r0, r1), kv_end, p8, seed, offset)
+        o[r0:r1], lse[r0:r1] = _finish(e, l, m, vh[:kv_end], z, r)
+    return o, lse
 
 
 def online_softmax_stats(logits, block: int):
