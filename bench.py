@@ -2,7 +2,8 @@
 """Benchmark of the attention hot path: one step = forward (fa_fwd) + backward (fa_bwd) of
 exact attention on one batch of seeded synthetic bf16 inputs, through the C ABI.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--dropout P]
+                    [--impl reference]
 
 Prints ONE JSON line (rank 0). ``value`` is whole-job attention TFLOP/s (fwd + bwd) with
 inputs resident in device memory; ``e2e`` is the same metric with pinned-host inputs copied in
@@ -11,6 +12,8 @@ independent replicas of the same workload, one per GPU (weak scaling); the only 
 are the barrier and the max-over-ranks of the timing.
 
 FLOP accounting: forward 4 B H N^2 d, backward 2.5x forward, both halved when causal.
+``--dropout P`` runs the same step with dropout probability P on the attention probabilities
+(fa_fwd_ex / fa_bwd_ex, a new Philox offset every step); the FLOP count is unchanged.
 ``--impl reference`` times the fp64 CPU oracle on the host instead, on bounded samples of the
 same workload.
 """
@@ -37,7 +40,8 @@ DEFAULT_WORKLOAD = "causal_train_b4h16n4096d128"
 L2_BYTES = 126 * 1024 * 1024
 FLUSH_BYTES = 512 * 1024 * 1024
 KERNEL_SOURCES = ["exact_io_aware_66_b200/csrc/fa_bwd.cuh", "exact_io_aware_66_b200/csrc/fa_fwd.cuh",
-                  "exact_io_aware_66_b200/csrc/sm100.cuh", "exact_io_aware_66_b200/csrc/fa_api.cu"]
+                  "exact_io_aware_66_b200/csrc/sm100.cuh", "exact_io_aware_66_b200/csrc/fa_api.cu",
+                  "exact_io_aware_66_b200/csrc/dropout.cuh"]
 
 
 def load_metric() -> str:
@@ -193,7 +197,7 @@ def oracle_threads() -> int:
     return len(os.sched_getaffinity(0))
 
 
-def oracle_head_step(x, w, heads, prefix: int | None = None):
+def oracle_head_step(x, w, heads, prefix: int | None = None, dropout: float = 0.0):
     """Oracle fwd+bwd of the given (b, h) heads, optionally restricted to the first `prefix`
     rows and keys (a self-contained sub-problem under the causal mask). Returns FLOPs done."""
     import numpy as np
@@ -203,25 +207,26 @@ def oracle_head_step(x, w, heads, prefix: int | None = None):
     n = w.N if prefix is None else prefix
     for b, h in heads:
         q, k, v = (x[t][b, h, :n].float().numpy().astype(np.float64) for t in ("q", "k", "v"))
+        dr = (dropout, 1, 0) if dropout > 0 else None
         if w.backward:
             do = x["do"][b, h, :n].float().numpy().astype(np.float64)
-            oracle.attention_backward(q, k, v, do, w.scale, w.causal)
+            oracle.attention_backward(q, k, v, do, w.scale, w.causal, dropout=dr)
         else:
-            oracle.attention_forward(q, k, v, w.scale, w.causal)
+            oracle.attention_forward(q, k, v, w.scale, w.causal, dropout=dr)
     f = 4.0 * n * n * w.d * (3.5 if w.backward else 1.0) * len(heads)
     return f / 2 if w.causal else f
 
 
-def cpu_baseline(w, x, budget_s: float = 12.0) -> dict:
+def cpu_baseline(w, x, budget_s: float = 12.0, dropout: float = 0.0) -> dict:
     heads_all = [(b, h) for b in range(w.B) for h in range(w.H)]
     t0 = time.perf_counter()
-    flops = oracle_head_step(x, w, heads_all[:1], prefix=min(w.N, 4096))
+    flops = oracle_head_step(x, w, heads_all[:1], prefix=min(w.N, 4096), dropout=dropout)
     one = time.perf_counter() - t0
     prefix = min(w.N, 4096)
     nh = max(1, min(len(heads_all), int(budget_s / max(one, 1e-3))))
     heads = heads_all[:nh]
     t0 = time.perf_counter()
-    flops = oracle_head_step(x, w, heads, prefix=prefix)
+    flops = oracle_head_step(x, w, heads, prefix=prefix, dropout=dropout)
     dt = time.perf_counter() - t0
     sample = (f"oracle fwd{'+bwd' if w.backward else ''} (fp64 NumPy) of {nh} of {len(heads_all)} "
               f"heads" + (f", first {prefix} rows/keys of each" if prefix < w.N else "")
@@ -245,12 +250,12 @@ def run_reference(args, w, world, rank):
     n = max(128, n // 128 * 128)
     heads = [(0, 0)]
     for _ in range(warm):
-        oracle_head_step(x, w, heads, prefix=n)
+        oracle_head_step(x, w, heads, prefix=n, dropout=args.dropout)
     t0 = time.perf_counter()
     flops = 0.0
     for s in range(steps):
         b, h = divmod(s % (w.B * w.H), w.H)
-        flops += oracle_head_step(x, w, [(b, h)], prefix=n)
+        flops += oracle_head_step(x, w, [(b, h)], prefix=n, dropout=args.dropout)
     dt = time.perf_counter() - t0
     value = flops / dt / 1e12
     sample = (f"per step: oracle fwd{'+bwd' if w.backward else ''} (fp64 NumPy) of one head, "
@@ -259,7 +264,7 @@ def run_reference(args, w, world, rank):
             "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": dt * 1000 / steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1), bf16-rounded, widened to fp64)",
-            "config": workload_config(w, world),
+            "config": workload_config(w, world, args.dropout),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -268,9 +273,11 @@ def run_reference(args, w, world, rank):
     return 0
 
 
-def workload_config(w, world) -> dict:
-    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+def workload_config(w, world, dropout: float = 0.0) -> dict:
+    return {"workload": w.name + (f"+dropout{dropout:g}" if dropout > 0 else ""),
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
             "pass": "fwd+bwd" if w.backward else "fwd", "scale": "1/sqrt(d)",
+            "dropout": dropout,
             "flops_per_step": w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": f"{FLUSH_BYTES >> 20} MiB buffer written before every timed step "
@@ -289,9 +296,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dropout", type=float, default=0.0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if not 0.0 <= args.dropout < 1.0:
+        ap.error("--dropout must be in [0, 1)")
     w = WORKLOADS[args.workload]
     world, rank, local = dist_setup()
     if args.impl == "reference":
@@ -312,7 +322,16 @@ def main():
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     stream = torch.cuda.current_stream(dev)
 
+    counter = [0]
+
     def step(q_, k_, v_, do_):
+        if args.dropout > 0:
+            dr = (args.dropout, 0x5EED, counter[0])  # a fresh Philox offset every step
+            counter[0] += 1
+            fa.fa_fwd_ex(q_, k_, v_, o, lse, w.causal, None, stream, dr)
+            if w.backward:
+                fa.fa_bwd_ex(q_, k_, v_, o, do_, lse, dq, dk, dv, ws, w.causal, None, stream, dr)
+            return
         fa.fa_fwd(q_, k_, v_, o, lse, w.causal, None, stream)
         if w.backward:
             fa.fa_bwd(q_, k_, v_, o, do_, lse, dq, dk, dv, ws, w.causal, None, stream)
@@ -362,7 +381,7 @@ def main():
     achieved = dom_flops / (avg_ms / 1e3) / 1e12 if dom_flops else None
     roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak if achieved else None,
-                "traffic": ncu_traffic(dom, w.name),
+                "traffic": ncu_traffic(dom, workload_config(w, world, args.dropout)["workload"]),
                 "peak_source": f"{peaks['source']} bf16 "
                                f"{'sustained' if ms_total > 1000 else 'burst'} (MEASURED_PEAKS.json)",
                 "per_launch_flops": dom_flops, "avg_launch_ms": avg_ms}
@@ -401,7 +420,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, x)
+        cpu = cpu_baseline(w, x, dropout=args.dropout)
 
     if rank == 0:
         line = {
@@ -410,7 +429,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1)" + (f" x{w.mult}" if w.mult != 1 else "")
                     + ", bf16), inputs resident in device memory",
-            "config": workload_config(w, world),
+            "config": workload_config(w, world, args.dropout),
             "fwd_tflops": w.fwd_flops() / (fwd_ms / 1e3) / 1e12 if fwd_ms else None,
             "bwd_tflops": (w.bwd_flops() / (bwd_ms / 1e3) / 1e12) if bwd_ms else None,
             "frac_of_peak": {"fwd+bwd": value / world / peaks["bf16_burst"],

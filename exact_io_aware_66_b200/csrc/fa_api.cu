@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -81,8 +82,8 @@ struct DeviceState {
   int* status = nullptr;  // device status word
   bool checked = false;   // compute capability verified
   bool is_sm100 = false;
-  bool fwd_attr[2][2] = {{false, false}, {false, false}};  // [d==128][causal]
-  bool bwd_attr[2][2] = {{false, false}, {false, false}};
+  bool fwd_attr[2][2][2] = {};  // [d==128][causal][dropout]: shared-memory attribute set
+  bool bwd_attr[2][2][2] = {};
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -189,6 +190,8 @@ struct Shape {
   int B, H, H_kv, N_q, N_kv, d;
   float scale;
   int mask;
+  bool dropout = false;     // set by apply_dropout for a drop probability that rounds above 0
+  fa::DropoutParams drop{};
   size_t q_bytes() const { return static_cast<size_t>(B) * H * N_q * d * 2; }
   size_t kv_bytes() const { return static_cast<size_t>(B) * H_kv * N_kv * d * 2; }
   size_t lse_bytes() const { return static_cast<size_t>(B) * H * N_q * 4; }
@@ -212,12 +215,29 @@ fa_status check_shape(const Shape& s) {
   return FA_OK;
 }
 
-template <int D, bool CAUSAL>
+// Dropout settings of the extended entry points (NULL: none). The drop probability is rounded
+// to p8 / 256, p8 = min(255, floor(256 p + 1/2)); p8 = 0 runs the kernels without dropout.
+fa_status apply_dropout(Shape& s, const fa_dropout* d) {
+  if (!d) return FA_OK;
+  if (!std::isfinite(d->p) || d->p < 0.f || d->p >= 1.f)
+    return set_err(FA_ERR_INVALID_ARG, "dropout probability %g not in [0, 1)", (double)d->p);
+  const int p8 = std::min(255, static_cast<int>(std::floor(256.0 * d->p + 0.5)));
+  if (p8 == 0) return FA_OK;
+  s.dropout = true;
+  s.drop.seed_lo = static_cast<uint32_t>(d->seed & 0xffffffffull);
+  s.drop.seed_hi = static_cast<uint32_t>(d->seed >> 32);
+  s.drop.offset = d->offset;
+  s.drop.add4 = static_cast<uint32_t>(256 - p8) * 0x01010101u;
+  s.drop.keep_scale = static_cast<float>(256.0 / (256 - p8));
+  return FA_OK;
+}
+
+template <int D, bool CAUSAL, bool DROPOUT>
 fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
                      float* lse, const Shape& s, cudaStream_t stream) {
   using L = fa::FwdLayout<D>;
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
-  bool& attr = ds->fwd_attr[D == 128][CAUSAL];
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, DROPOUT>;
+  bool& attr = ds->fwd_attr[D == 128][CAUSAL][DROPOUT];
   if (!attr) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -250,6 +270,7 @@ fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* 
   p.n_qblocks = (s.N_q + 255) / 256;
   p.scale = s.scale;
   p.scale_log2 = s.scale * 1.4426950408889634f;
+  p.drop = s.drop;
   const long long grid = 1LL * p.n_qblocks * BH;
   if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
   ProfileScope prof(0, stream);
@@ -259,13 +280,13 @@ fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* 
   return FA_OK;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DROPOUT>
 fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* v, const void* o,
                      const void* dO, const float* lse, void* dq, void* dk, void* dv,
                      void* workspace, const Shape& s, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
-  auto kern = fa::fa_bwd_main<D, CAUSAL>;
-  bool& attr = ds->bwd_attr[D == 128][CAUSAL];
+  auto kern = fa::fa_bwd_main<D, CAUSAL, DROPOUT>;
+  bool& attr = ds->bwd_attr[D == 128][CAUSAL][DROPOUT];
   if (!attr) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -332,6 +353,7 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   }
   p.scale = s.scale;
   p.scale_log2 = s.scale * 1.4426950408889634f;
+  p.drop = s.drop;
   const long long grid = 1LL * p.n_kv * BHkv;
   if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
   {
@@ -353,14 +375,30 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   return FA_OK;
 }
 
+template <int D, bool CAUSAL>
+fa_status fwd_dispatch_d(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
+                         float* lse, const Shape& s, cudaStream_t stream) {
+  return s.dropout ? launch_fwd<D, CAUSAL, true>(ds, q, k, v, o, lse, s, stream)
+                   : launch_fwd<D, CAUSAL, false>(ds, q, k, v, o, lse, s, stream);
+}
+
 fa_status fwd_dispatch(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
                        float* lse, const Shape& s, cudaStream_t stream) {
   const bool causal = s.mask != 0;
   if (s.d == 64)
-    return causal ? launch_fwd<64, true>(ds, q, k, v, o, lse, s, stream)
-                  : launch_fwd<64, false>(ds, q, k, v, o, lse, s, stream);
-  return causal ? launch_fwd<128, true>(ds, q, k, v, o, lse, s, stream)
-                : launch_fwd<128, false>(ds, q, k, v, o, lse, s, stream);
+    return causal ? fwd_dispatch_d<64, true>(ds, q, k, v, o, lse, s, stream)
+                  : fwd_dispatch_d<64, false>(ds, q, k, v, o, lse, s, stream);
+  return causal ? fwd_dispatch_d<128, true>(ds, q, k, v, o, lse, s, stream)
+                : fwd_dispatch_d<128, false>(ds, q, k, v, o, lse, s, stream);
+}
+
+template <int D, bool CAUSAL>
+fa_status bwd_dispatch_d(DeviceState* ds, const void* q, const void* k, const void* v,
+                         const void* o, const void* dO, const float* lse, void* dq, void* dk,
+                         void* dv, void* workspace, const Shape& s, cudaStream_t stream) {
+  return s.dropout
+             ? launch_bwd<D, CAUSAL, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream)
+             : launch_bwd<D, CAUSAL, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
 }
 
 fa_status bwd_dispatch(DeviceState* ds, const void* q, const void* k, const void* v, const void* o,
@@ -368,10 +406,10 @@ fa_status bwd_dispatch(DeviceState* ds, const void* q, const void* k, const void
                        void* workspace, const Shape& s, cudaStream_t stream) {
   const bool causal = s.mask != 0;
   if (s.d == 64)
-    return causal ? launch_bwd<64, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream)
-                  : launch_bwd<64, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
-  return causal ? launch_bwd<128, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream)
-                : launch_bwd<128, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
+    return causal ? bwd_dispatch_d<64, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream)
+                  : bwd_dispatch_d<64, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
+  return causal ? bwd_dispatch_d<128, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream)
+                : bwd_dispatch_d<128, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
 }
 
 // Argument checks of the forward (nothing is launched when one fails), then the launch.
@@ -464,7 +502,7 @@ struct NoAllocDevice {
   bool ready = false;
   void* scratch = nullptr;  // device address of g_noalloc_scratch on this device
   int* status = nullptr;    // device address of g_noalloc_status on this device
-  bool bwd_attr[2][2] = {{false, false}, {false, false}};
+  bool bwd_attr[2][2][2] = {};
 };
 NoAllocDevice g_noalloc[kMaxDevices];
 
@@ -483,10 +521,13 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 }
 
 fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
-                    const fa_attn_shape* shape, void* stream) {
+                    const fa_attn_shape* shape, const fa_dropout* dropout, void* stream) {
   g_err[0] = '\0';
   if (!shape) return set_err(FA_ERR_INVALID_ARG, "null shape");
-  return fwd_checked(q, k, v, o, lse, from_public(shape), stream);
+  Shape s = from_public(shape);
+  const fa_status st = apply_dropout(s, dropout);
+  if (st != FA_OK) return st;
+  return fwd_checked(q, k, v, o, lse, s, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -514,11 +555,14 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
 
 fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dO,
                     const float* lse, void* dq, void* dk, void* dv, void* workspace,
-                    size_t workspace_bytes, const fa_attn_shape* shape, void* stream) {
+                    size_t workspace_bytes, const fa_attn_shape* shape,
+                    const fa_dropout* dropout, void* stream) {
   g_err[0] = '\0';
   if (!shape) return set_err(FA_ERR_INVALID_ARG, "null shape");
-  return bwd_checked(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes,
-                     from_public(shape), stream);
+  Shape s = from_public(shape);
+  const fa_status st = apply_dropout(s, dropout);
+  if (st != FA_OK) return st;
+  return bwd_checked(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, s, stream);
 }
 
 fa_status fa_profile_enable(int on) {

@@ -24,6 +24,7 @@
 //      The final dK (times scale) and dV are stored with TMA.
 //   3. fa_bwd_dq_convert: dQ = bf16(dQ_acc).
 #pragma once
+#include "dropout.cuh"
 #include "fa_fwd.cuh"
 #include "sm100.cuh"
 
@@ -161,9 +162,10 @@ struct BwdParams {
   int group;       // key/value heads per scheduling group
   float scale;
   float scale_log2;
+  DropoutParams drop;  // read only by the DROPOUT instantiations
 };
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DROPOUT>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -265,6 +267,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                              (k0 + 128 > p.N_kv);
       uint32_t pk[16], dsk[16];
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      // Dropout keep bits of this key for the 32 queries: the quad's four lanes (keys 4J..4J+3)
+      // run two generator calls each (blocks of queries 4n..4n+3 for n = lane%4 and 4 + lane%4),
+      // transpose each block's bytes so that word t holds key t's four bytes, and swap words:
+      // kbits[h][g] then holds queries qbase + 16h + 4g + (0..3) of this key.
+      uint32_t kbits[2][4];
+      if constexpr (DROPOUT) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t wv[4] = {static_cast<uint32_t>(key) >> 2,
+                            static_cast<uint32_t>((qbase >> 2) + 4 * h + (lane & 3)),
+                            static_cast<uint32_t>(q_head(i)), p.drop.offset};
+          philox4x32_10(wv, p.drop.seed_lo, p.drop.seed_hi);
+          byte_transpose(wv, kbits[h]);
+          quad_transpose(kbits[h], lane);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) kbits[h][g] = keep_bytes(kbits[h][g], p.drop.add4);
+        }
+      }
+      const uint64_t rk2 = f2_pack(p.drop.keep_scale, p.drop.keep_scale);
 #pragma unroll
       for (int c = 0; c < 32; c += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);  // -lse * log2(e)
@@ -274,12 +295,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         f2_unpack(f2_fma(f2_pack_u(s[c + 2], s[c + 3]), sl2x2, f2_pack(l4.z, l4.w)), a[2], a[3]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) pr[e] = ex2_approx(a[e]);
-        f2_unpack(f2_mul(f2_pack(pr[0], pr[1]),
-                         f2_sub(f2_pack_u(dp[c], dp[c + 1]), f2_pack(d4.x, d4.y))),
-                  dsr[0], dsr[1]);
-        f2_unpack(f2_mul(f2_pack(pr[2], pr[3]),
-                         f2_sub(f2_pack_u(dp[c + 2], dp[c + 3]), f2_pack(d4.z, d4.w))),
-                  dsr[2], dsr[3]);
+        if constexpr (!DROPOUT) {
+          f2_unpack(f2_mul(f2_pack(pr[0], pr[1]),
+                           f2_sub(f2_pack_u(dp[c], dp[c + 1]), f2_pack(d4.x, d4.y))),
+                    dsr[0], dsr[1]);
+          f2_unpack(f2_mul(f2_pack(pr[2], pr[3]),
+                           f2_sub(f2_pack_u(dp[c + 2], dp[c + 3]), f2_pack(d4.z, d4.w))),
+                    dsr[2], dsr[3]);
+        } else {
+          // dS = P o (r Z o dP - D); the P fed to the dV MMA is Z o P (r is applied to dV at
+          // the end)
+          const uint32_t kb = kbits[c / 16][(c / 4) & 3];
+          const uint32_t m0 = elem_mask<0>(kb), m1 = elem_mask<1>(kb);
+          const uint32_t m2 = elem_mask<2>(kb), m3 = elem_mask<3>(kb);
+          f2_unpack(f2_mul(f2_pack(pr[0], pr[1]),
+                           f2_fma(f2_pack_u(dp[c] & m0, dp[c + 1] & m1), rk2,
+                                  f2_pack(-d4.x, -d4.y))),
+                    dsr[0], dsr[1]);
+          f2_unpack(f2_mul(f2_pack(pr[2], pr[3]),
+                           f2_fma(f2_pack_u(dp[c + 2] & m2, dp[c + 3] & m3), rk2,
+                                  f2_pack(-d4.z, -d4.w))),
+                    dsr[2], dsr[3]);
+          pr[0] = __uint_as_float(__float_as_uint(pr[0]) & m0);
+          pr[1] = __uint_as_float(__float_as_uint(pr[1]) & m1);
+          pr[2] = __uint_as_float(__float_as_uint(pr[2]) & m2);
+          pr[3] = __uint_as_float(__float_as_uint(pr[3]) & m3);
+        }
         if (need_mask) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -312,7 +353,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       // warpgroup 0 stores dV (stage-0 Q/dO space), warpgroup 1 stores dK * scale (stage 1)
       const uint32_t tcol = w == 0 ? L::tDV : L::tDK;
-      const float mul = w == 0 ? 1.0f : p.scale;
+      const float mul = w == 0 ? (DROPOUT ? p.drop.keep_scale : 1.0f) : p.scale;
       const int region = L::kQ + w * 2 * L::kQTile;
       uint8_t* stage = gbase + region;
 #pragma unroll

@@ -22,6 +22,7 @@
 // MMA issue order per key tile j: PV0(j), S0(j+1), PV1(j), S1(j+1) — while softmax 0 works on
 // S0(j+1) the tensor core runs PV1(j) and S1(j+1), and vice versa.
 #pragma once
+#include "dropout.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -30,9 +31,17 @@ constexpr int kFwdThreads = 512;
 // Register split (setmaxnreg): softmax warps 0-7, epilogue warps 8-11, MMA/TMA warps 12-15.
 // setmaxnreg.inc waits until the decrements have freed enough registers, so the split must add
 // up to exactly the launch allocation (512 threads x 128 registers; checked on the host).
-constexpr uint32_t kFwdRegSoftmax = 176, kFwdRegEpilogue = 64, kFwdRegMma = 96;
-static_assert(256 * kFwdRegSoftmax + 128 * kFwdRegEpilogue + 128 * kFwdRegMma == kFwdThreads * 128,
-              "forward register split must equal the launch allocation");
+// The d = 64 dropout variant moves 16 registers per thread from the MMA/TMA warps (whose d = 64
+// issue loop needs fewer) to the softmax warps, which also run the random-number generator.
+template <int D, bool DROPOUT>
+struct FwdRegs {
+  static constexpr bool kShift = DROPOUT && D == 64;
+  static constexpr uint32_t kSoftmax = kShift ? 184 : 176;
+  static constexpr uint32_t kEpilogue = 64;
+  static constexpr uint32_t kMma = kShift ? 80 : 96;
+  static_assert(256 * kSoftmax + 128 * kEpilogue + 128 * kMma == kFwdThreads * 128,
+                "forward register split must equal the launch allocation");
+};
 // Running-max update threshold, log2 units (exponentials stay below 2^8 between updates).
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -73,6 +82,7 @@ struct FwdParams {
   int n_qblocks;    // ceil(N / 256)
   float scale;      // softmax scale
   float scale_log2; // scale * log2(e)
+  DropoutParams drop;  // read only by the DROPOUT instantiations
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -106,7 +116,7 @@ __device__ __forceinline__ void fail(int* status, volatile int* abort_flag, int 
   atomicExch(status, code);
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DROPOUT>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -174,7 +184,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (warp < 8) {
     // ------------------------------------------------------------------ softmax ----------
-    setmaxnreg_inc<kFwdRegSoftmax>();
+    setmaxnreg_inc<FwdRegs<D, DROPOUT>::kSoftmax>();
     const int t = warp >> 2;
     const int row = threadIdx.x & 127;
     const uint32_t tS = tmem + t * 128 + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -228,15 +238,45 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint64_t sl2x2 = f2_pack(sl2, sl2), nbx2 = f2_pack(nb, nb);
       uint64_t lsum[4] = {0, 0, 0, 0}, rsum[4] = {0, 0, 0, 0};  // (0.f, 0.f) pairs
       uint32_t pk[64];
+      if constexpr (!DROPOUT) {
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        float a0, a1;
-        f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, nbx2), a0, a1);
-        const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
-        const uint32_t w = pack_bf16x2(e0, e1);
-        pk[c / 2] = w;
-        lsum[(c >> 1) & 3] = f2_add(lsum[(c >> 1) & 3], f2_pack(e0, e1));
-        rsum[(c >> 1) & 3] = f2_add(rsum[(c >> 1) & 3], f2_pack_u(w << 16, w & 0xffff0000u));
+        for (int c = 0; c < 128; c += 2) {
+          float a0, a1;
+          f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, nbx2), a0, a1);
+          const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
+          const uint32_t w = pack_bf16x2(e0, e1);
+          pk[c / 2] = w;
+          lsum[(c >> 1) & 3] = f2_add(lsum[(c >> 1) & 3], f2_pack(e0, e1));
+          rsum[(c >> 1) & 3] = f2_add(rsum[(c >> 1) & 3], f2_pack_u(w << 16, w & 0xffff0000u));
+        }
+      } else {
+        // Dropout: the sums l, lr take every weight; the P handed to the PV MMA keeps only the
+        // kept ones (the keep scale is applied with 1/lr in the epilogue). Keys are taken 16
+        // at a time: the quad's four lanes each run one generator call (one 4 x 4 block) and
+        // swap words so that each lane holds its own row's bytes for the 16 keys.
+#pragma unroll
+        for (int mc = 0; mc < 8; ++mc) {
+          uint32_t kw[4] = {static_cast<uint32_t>(32 * j + 4 * mc + (lane & 3)),
+                            static_cast<uint32_t>(q_row) >> 2, static_cast<uint32_t>(bh),
+                            p.drop.offset};
+          philox4x32_10(kw, p.drop.seed_lo, p.drop.seed_hi);
+          quad_transpose(kw, lane);  // kw[g]: bytes of keys 16 mc + 4 g + (0..3), this row
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t kb = keep_bytes(kw[g], p.drop.add4);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int c = 16 * mc + 4 * g + 2 * h;
+              float a0, a1;
+              f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, nbx2), a0, a1);
+              const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
+              const uint32_t w = pack_bf16x2(e0, e1);
+              pk[c / 2] = w & (h == 0 ? pair_mask<0>(kb) : pair_mask<1>(kb));
+              lsum[(c >> 1) & 3] = f2_add(lsum[(c >> 1) & 3], f2_pack(e0, e1));
+              rsum[(c >> 1) & 3] = f2_add(rsum[(c >> 1) & 3], f2_pack_u(w << 16, w & 0xffff0000u));
+            }
+          }
+        }
       }
       {
         const uint64_t ls = f2_add(f2_add(lsum[0], lsum[1]), f2_add(lsum[2], lsum[3]));
@@ -282,7 +322,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           l > 0.f ? (m * sl2 + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
   } else if (warp < 12) {
     // ----------------------------------------------------------------- epilogue ----------
-    setmaxnreg_dec<kFwdRegEpilogue>();
+    setmaxnreg_dec<FwdRegs<D, DROPOUT>::kEpilogue>();
     const int row = threadIdx.x - 256;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
@@ -300,7 +340,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       tc_fence_after();
       const float lr_row = s_rowl[t * 128 + row];
-      const float inv_l = lr_row > 0.f ? 1.0f / lr_row : 0.f;
+      float inv_l = lr_row > 0.f ? 1.0f / lr_row : 0.f;
+      if constexpr (DROPOUT) inv_l = lr_row > 0.f ? p.drop.keep_scale / lr_row : 0.f;
       const bool empty_tile = n_t[t] == 0;  // no PV ever wrote this O accumulator
       const uint32_t tO = tmem + 256 + t * D + lane_off;
       uint8_t* stage = gbase + L::kQ + t * L::kTileBytes;
@@ -340,7 +381,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     if (lane == 0) bulk_wait_group_read0();
   } else {
-    setmaxnreg_dec<kFwdRegMma>();
+    setmaxnreg_dec<FwdRegs<D, DROPOUT>::kMma>();
     if (warp == 12 && lane == 0) {
       // ------------------------------------------------------------------ MMA -------------
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);

@@ -38,9 +38,9 @@ SIGNATURES = {
     "fa_kernel_name": (ctypes.c_char_p, [_I]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_selftest_timeout": (_I, [_I, _P]),
-    "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P]),
+    "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "fa_bwd_ex_workspace_size": (_Z, [_P]),
-    "fa_bwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
+    "fa_bwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P, _P]),
 }
 
 # fa_mask values
@@ -52,6 +52,19 @@ class FaAttnShape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int),
                 ("N_q", ctypes.c_int), ("N_kv", ctypes.c_int), ("d", ctypes.c_int),
                 ("scale", ctypes.c_float), ("mask", ctypes.c_int)]
+
+
+class FaDropout(ctypes.Structure):
+    """struct fa_dropout of include/fa.h."""
+    _fields_ = [("p", ctypes.c_float), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint)]
+
+
+def _dropout_arg(dropout):
+    """None, or (p, seed, offset) -> a pointer to an fa_dropout (None stays a NULL pointer)."""
+    if dropout is None:
+        return None
+    p, seed, offset = dropout
+    return ctypes.byref(FaDropout(float(p), int(seed), int(offset)))
 
 
 def mask_code(causal) -> int:
@@ -226,16 +239,19 @@ def _shape(q, k, v, causal, scale) -> FaAttnShape:
     return FaAttnShape(B, H, H_kv, N_q, N_kv, d, scale, mask_code(causal))
 
 
-def fa_fwd_ex(q, k, v, o, lse, causal=False, scale: float | None = None, stream=None):
+def fa_fwd_ex(q, k, v, o, lse, causal=False, scale: float | None = None, stream=None,
+              dropout=None):
     """Forward for q [B,H,N_q,d] and k, v [B,H_kv,N_kv,d] (H a multiple of H_kv) into
-    caller-allocated o (like q) and lse (fp32 [B,H,N_q]); causal as in mask_code."""
+    caller-allocated o (like q) and lse (fp32 [B,H,N_q]); causal as in mask_code; dropout None
+    or (p, seed, offset) as in include/fa.h."""
     s = _shape(q, k, v, causal, scale)
     if _dims(o) != (s.B, s.H, s.N_q, s.d):
         raise ValueError("o shape mismatch")
     if tuple(lse.shape) != (s.B, s.H, s.N_q):
         raise ValueError("lse must be [B, H, N_q]")
     ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(lse, "lse", torch.float32)]
-    _check("fa_fwd_ex", lib().fa_fwd_ex(*ptrs, ctypes.byref(s), _stream_handle(stream)))
+    _check("fa_fwd_ex", lib().fa_fwd_ex(*ptrs, ctypes.byref(s), _dropout_arg(dropout),
+                                        _stream_handle(stream)))
 
 
 def fa_bwd_ex_workspace_size(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int,
@@ -246,9 +262,10 @@ def fa_bwd_ex_workspace_size(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: 
 
 
 def fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, causal=False,
-              scale: float | None = None, stream=None):
+              scale: float | None = None, stream=None, dropout=None):
     """Backward for the shapes of fa_fwd_ex into caller-allocated dq (like q), dk, dv (like k)
-    with a caller-owned workspace of at least fa_bwd_ex_workspace_size bytes."""
+    with a caller-owned workspace of at least fa_bwd_ex_workspace_size bytes; dropout as given
+    to the forward that produced o and lse."""
     s = _shape(q, k, v, causal, scale)
     for t, n in ((o, "o"), (do, "do"), (dq, "dq")):
         if _dims(t) != (s.B, s.H, s.N_q, s.d):
@@ -264,28 +281,30 @@ def fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, causal=False,
             _req(lse, "lse", torch.float32), _req(dq, "dq"), _req(dk, "dk"), _req(dv, "dv")]
     wbytes = workspace.numel() * workspace.element_size()
     _check("fa_bwd_ex", lib().fa_bwd_ex(*ptrs, workspace.data_ptr(), wbytes, ctypes.byref(s),
-                                        _stream_handle(stream)))
+                                        _dropout_arg(dropout), _stream_handle(stream)))
 
 
-def attention_forward(q, k, v, causal=False, scale: float | None = None, stream=None):
+def attention_forward(q, k, v, causal=False, scale: float | None = None, stream=None,
+                      dropout=None):
     """Returns (o, lse) for bf16 CUDA tensors q [B, H, N_q, d] and k, v [B, H_kv, N_kv, d]
-    (H_kv = H and N_kv = N_q in the square case); causal as in mask_code."""
+    (H_kv = H and N_kv = N_q in the square case); causal as in mask_code; dropout None or
+    (p, seed, offset)."""
     B, H, N, d = _dims(q)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    fa_fwd_ex(q, k, v, o, lse, causal, scale, stream)
+    fa_fwd_ex(q, k, v, o, lse, causal, scale, stream, dropout)
     return o, lse
 
 
 def attention_backward(q, k, v, o, do, lse, causal=False, scale: float | None = None,
-                       stream=None, workspace=None):
-    """Returns (dq, dk, dv) for the shapes of attention_forward. Allocates the workspace
-    unless one is given."""
+                       stream=None, workspace=None, dropout=None):
+    """Returns (dq, dk, dv) for the shapes of attention_forward (dropout as given to it).
+    Allocates the workspace unless one is given."""
     B, H, N, d = _dims(q)
     _, H_kv, N_kv, _ = _dims(k)
     if workspace is None:
         workspace = torch.empty(fa_bwd_ex_workspace_size(B, H, H_kv, N, N_kv, d, causal),
                                 dtype=torch.uint8, device=q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, causal, scale, stream)
+    fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, causal, scale, stream, dropout)
     return dq, dk, dv

@@ -73,19 +73,38 @@ typedef struct {
   int mask;    /* an fa_mask value */
 } fa_attn_shape;
 
-/* Forward for an fa_attn_shape (fa_fwd is the case H_kv = H, N_q = N_kv = N). The pages define
- * the square, equal-head case; these shapes apply the same definition with the mask above. */
+/* Dropout on the attention probabilities, the pass that "How FlashAttention Actually Works"
+ * ("The GPU Memory Wall: HBM vs. SRAM") places between the softmax and the product with V.
+ * Inverted dropout: each entry of P is kept with probability 1 - p8/256 and scaled by
+ * 256/(256 - p8), where p8 = min(255, floor(256 p + 1/2)); lse stays that of the undropped
+ * softmax. No mask is stored: the forward and the backward regenerate the same decisions from
+ * Philox4x32-10 (Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11) with
+ * counter (j/4, i/4, b*H + h, offset) and key (seed low word, seed high word) for query i and
+ * key j of query head h; the entry's byte is byte (j mod 4) of output word (i mod 4), and the
+ * entry is kept iff that byte >= p8. Pass the same settings to the forward and the backward.
+ * A NULL fa_dropout pointer, or p8 = 0, means no dropout. */
+typedef struct {
+  float p;                 /* drop probability, in [0, 1) */
+  unsigned long long seed; /* Philox key */
+  unsigned int offset;     /* Philox counter word 3: vary it between calls that share a seed */
+} fa_dropout;
+
+/* Forward for an fa_attn_shape (fa_fwd is the case H_kv = H, N_q = N_kv = N, no dropout). The
+ * pages define the square, equal-head case; these shapes apply the same definition with the
+ * mask above. dropout: NULL or the settings above (FA_ERR_INVALID_ARG for p outside [0, 1)). */
 fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
-                    const fa_attn_shape* shape, void* stream);
+                    const fa_attn_shape* shape, const fa_dropout* dropout, void* stream);
 
 /* Workspace bytes fa_bwd_ex needs (fp32 dQ accumulator and row terms for B*H*N_q rows); 0 for an
  * invalid shape. */
 size_t fa_bwd_ex_workspace_size(const fa_attn_shape* shape);
 
-/* Backward for an fa_attn_shape; arguments as fa_bwd. */
+/* Backward for an fa_attn_shape; arguments as fa_bwd, and dropout as given to fa_fwd_ex for
+ * the o and lse passed here. */
 fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dO,
                     const float* lse, void* dq, void* dk, void* dv, void* workspace,
-                    size_t workspace_bytes, const fa_attn_shape* shape, void* stream);
+                    size_t workspace_bytes, const fa_attn_shape* shape,
+                    const fa_dropout* dropout, void* stream);
 
 /* Forward. Writes o (bf16 [B,H,N,d]) and lse (fp32 [B,H,N]).
  * scale: the softmax scale (finite, > 0), normally 1/sqrt(d). causal: 0 or 1.

@@ -4,6 +4,7 @@ Tolerances (fixed numbers, never loosened per case):
   forward O:   max-abs <= 1e-2 and mean-abs <= 1e-3 against the fp64 oracle
   lse:         max-abs <= 1e-3
   dQ, dK, dV:  max-abs error / max-abs of the oracle's tensor <= 2e-2, per tensor
+  with dropout: the O bounds times the keep scale r = 256 / (256 - p8) (see assert_fwd_ok)
 
 O is returned in bf16, whose spacing is 2^-5 on [4, 8): rounding the exact value alone can
 move it by up to 1.56e-2 there, more than 1e-2. Such "format-limited" elements (|O_ref| >= 4)
@@ -51,11 +52,14 @@ def fwd_errors(o_gpu, lse_gpu, o_ref, lse_ref) -> dict:
             "o_ref_absmax": float(np.abs(o_ref).max()) if o_ref.size else 0.0}
 
 
-def assert_fwd_ok(err: dict, what: str = ""):
+def assert_fwd_ok(err: dict, what: str = "", keep_scale: float = 1.0):
+    """keep_scale: with dropout, the kept weights (and so the rounding errors of P and of O) are
+    multiplied by r = 256 / (256 - p8); the O bounds are multiplied by the same r."""
     print(f"[parity] {what}: {err}")
-    assert err["o_max_in_range"] <= TOL_O_MAX, f"{what} O max-abs {err['o_max_in_range']:.3e}"
+    tol_max, tol_mean = TOL_O_MAX * keep_scale, TOL_O_MEAN * keep_scale
+    assert err["o_max_in_range"] <= tol_max, f"{what} O max-abs {err['o_max_in_range']:.3e}"
     assert err["format_ulps"] <= 1.0, f"{what} format-limited O off by {err['format_ulps']:.2f} ulp"
-    assert err["o_mean"] <= TOL_O_MEAN, f"{what} O mean-abs {err['o_mean']:.3e}"
+    assert err["o_mean"] <= tol_mean, f"{what} O mean-abs {err['o_mean']:.3e}"
     assert err["lse_max"] <= TOL_LSE, f"{what} lse max-abs {err['lse_max']:.3e}"
 
 

@@ -122,11 +122,11 @@ def test_selftest_timeout_rejects_bad_limit_without_gpu(lib):
 def _fwd_ex_raw(lib, B=1, H=2, H_kv=1, N_q=100, N_kv=300, d=64, scale=0.125, mask=2, o=1 << 20,
                 lse=2 << 20):
     s = fa.FaAttnShape(B, H, H_kv, N_q, N_kv, d, scale, mask)
-    return lib.fa_fwd_ex(16, 1 << 16, 2 << 16, o, lse, ctypes.byref(s), None)
+    return lib.fa_fwd_ex(16, 1 << 16, 2 << 16, o, lse, ctypes.byref(s), None, None)
 
 
 def test_fwd_ex_validation_without_gpu(lib):
-    assert lib.fa_fwd_ex(16, 32, 48, 1 << 20, 2 << 20, None, None) == 1  # null shape
+    assert lib.fa_fwd_ex(16, 32, 48, 1 << 20, 2 << 20, None, None, None) == 1  # null shape
     assert _fwd_ex_raw(lib, H=3, H_kv=2) == 1  # H not a multiple of H_kv
     assert "multiple" in fa.fa_last_error_string()
     assert _fwd_ex_raw(lib, mask=3) == 1
@@ -154,3 +154,12 @@ def test_mask_code():
     assert fa.mask_code("bottom_right") == 2
     with pytest.raises(ValueError):
         fa.mask_code("diagonal")
+
+
+def test_dropout_validation_without_gpu(lib):
+    s = fa.FaAttnShape(1, 2, 1, 100, 300, 64, 0.125, 2)
+    for p in (1.0, -0.1, float("nan")):
+        d = fa.FaDropout(p, 1, 0)
+        assert lib.fa_fwd_ex(16, 1 << 16, 2 << 16, 1 << 20, 2 << 20, ctypes.byref(s),
+                             ctypes.byref(d), None) == 1
+        assert "dropout" in fa.fa_last_error_string()
