@@ -74,3 +74,39 @@ def assert_grad_ok(g_gpu, g_ref, what: str):
     r = grad_rel_error(g_gpu, g_ref)
     assert r <= TOL_GRAD_REL, f"{what} relative max-norm error {r:.3e}"
     return r
+
+
+# ------------------------------------------------------------------------------------------
+# FP8 forward bounds
+# ------------------------------------------------------------------------------------------
+def fp8_bounds(s_rows: np.ndarray, v: np.ndarray, o_ref: np.ndarray):
+    """Error bounds of an FP8 forward output row block against the exact O of the decoded inputs.
+
+    s_rows: [r, n] fp64 scores (masked entries -inf), v: [n, d] decoded V, o_ref: [r, d].
+    The kernel rounds each weight e_j = exp(s_j - m) to E4M3, with m its running max, at most 8
+    log2-units below the row max, and normalises by the sum of the rounded weights, so exactly
+        O - O* = sum_j (e~_j - e_j)(v_j - O*) / sum_j e~_j.
+    E4M3 rounding moves a weight by at most half a unit in the last place: 2^-4 e_j in the
+    normal range (e_j >= 2^-6), and min(e_j, 2^-10) in the subnormal range (spacing 2^-9).
+    With e^_j = exp(s_j - max s) (e_j = 2^delta e^_j, delta in [0, 8], so e^_j >= 2^-6 implies
+    the normal range) and L^ = sum_j e^_j, dividing through by 2^delta:
+        err_j      = 2^-4 e^_j + [e^_j < 2^-6] min(e^_j, 2^-10)
+        max bound  = sum_j err_j |v_j - O*| / (L^ - sum_j err_j)
+                     + 2^-8 |O*| (bf16 output rounding) + 1e-5 max|v| (fp32 arithmetic)
+        mean bound = sqrt(2/pi) 2^-4 / sqrt(3) sqrt(sum_j (e^_j / L^)^2 (v_j - O*)^2)
+    the second being the mean absolute value of the sum when the relative rounding errors are
+    independent and uniform (standard deviation 2^-4 / sqrt 3). Returns (max_bound [r, d],
+    mean_bound [r, d], ok) with ok False where the max bound's denominator is not positive."""
+    mx = np.max(s_rows, axis=1, keepdims=True)
+    mx = np.where(np.isfinite(mx), mx, 0.0)
+    eh = np.exp(s_rows - mx)  # masked entries: exp(-inf) = 0
+    L = eh.sum(axis=1, keepdims=True)
+    err = 2.0 ** -4 * eh + np.where(eh < 2.0 ** -6, np.minimum(eh, 2.0 ** -10), 0.0)
+    dev = np.abs(v[None, :, :] - o_ref[:, None, :])  # [r, n, d]
+    num = np.einsum("rn,rnd->rd", err, dev)
+    den = L - err.sum(axis=1, keepdims=True)
+    ok = den[:, 0] > 0
+    maxb = num / np.where(den > 0, den, np.inf) + 2.0 ** -8 * np.abs(o_ref) + 1e-5 * np.abs(v).max()
+    w2 = (eh / np.where(L > 0, L, 1.0)) ** 2
+    meanb = np.sqrt(2 / np.pi) * 2.0 ** -4 / np.sqrt(3) * np.sqrt(np.einsum("rn,rnd->rd", w2, dev ** 2))
+    return maxb, meanb, ok
