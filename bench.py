@@ -12,7 +12,9 @@ independent replicas of the same workload, one per GPU (weak scaling); the only 
 are the barrier and the max-over-ranks of the timing.
 
 FLOP accounting: forward 4 B H N^2 d, backward 2.5x forward, both halved when causal.
-``--dropout P`` runs the same step with dropout probability P on the attention probabilities
+``--fp8`` times the FP8 (E4M3) forward of the workload instead (fa_fwd_fp8, forward only, its
+FLOPs counted as for bf16, the roofline against twice the measured bf16 peak — the nominal
+FP8/bf16 ratio). ``--dropout P`` runs the same step with dropout probability P on the attention probabilities
 (fa_fwd_ex / fa_bwd_ex, a new Philox offset every step); the FLOP count is unchanged.
 ``--impl reference`` times the fp64 CPU oracle on the host instead, on bounded samples of the
 same workload.
@@ -41,7 +43,8 @@ L2_BYTES = 126 * 1024 * 1024
 FLUSH_BYTES = 512 * 1024 * 1024
 KERNEL_SOURCES = ["exact_io_aware_66_b200/csrc/fa_bwd.cuh", "exact_io_aware_66_b200/csrc/fa_fwd.cuh",
                   "exact_io_aware_66_b200/csrc/sm100.cuh", "exact_io_aware_66_b200/csrc/fa_api.cu",
-                  "exact_io_aware_66_b200/csrc/dropout.cuh"]
+                  "exact_io_aware_66_b200/csrc/dropout.cuh",
+                  "exact_io_aware_66_b200/csrc/fa_fwd_fp8.cuh"]
 
 
 def load_metric() -> str:
@@ -197,7 +200,8 @@ def oracle_threads() -> int:
     return len(os.sched_getaffinity(0))
 
 
-def oracle_head_step(x, w, heads, prefix: int | None = None, dropout: float = 0.0):
+def oracle_head_step(x, w, heads, prefix: int | None = None, dropout: float = 0.0,
+                     fp8: bool = False):
     """Oracle fwd+bwd of the given (b, h) heads, optionally restricted to the first `prefix`
     rows and keys (a self-contained sub-problem under the causal mask). Returns FLOPs done."""
     import numpy as np
@@ -205,6 +209,14 @@ def oracle_head_step(x, w, heads, prefix: int | None = None, dropout: float = 0.
     import oracle
 
     n = w.N if prefix is None else prefix
+    if fp8:
+        from oracle.fp8 import attention_forward_fp8
+
+        for b, h in heads:
+            codes = [x[t][b, h, :n].view(torch.uint8).numpy() for t in ("q8", "k8", "v8")]
+            attention_forward_fp8(*codes, *x["descale"], w.scale, w.causal)
+        f = 4.0 * n * n * w.d * len(heads)
+        return f / 2 if w.causal else f
     for b, h in heads:
         q, k, v = (x[t][b, h, :n].float().numpy().astype(np.float64) for t in ("q", "k", "v"))
         dr = (dropout, 1, 0) if dropout > 0 else None
@@ -217,18 +229,20 @@ def oracle_head_step(x, w, heads, prefix: int | None = None, dropout: float = 0.
     return f / 2 if w.causal else f
 
 
-def cpu_baseline(w, x, budget_s: float = 12.0, dropout: float = 0.0) -> dict:
+def cpu_baseline(w, x, budget_s: float = 12.0, dropout: float = 0.0, fp8: bool = False) -> dict:
     heads_all = [(b, h) for b in range(w.B) for h in range(w.H)]
     t0 = time.perf_counter()
-    flops = oracle_head_step(x, w, heads_all[:1], prefix=min(w.N, 4096), dropout=dropout)
+    flops = oracle_head_step(x, w, heads_all[:1], prefix=min(w.N, 4096), dropout=dropout, fp8=fp8)
     one = time.perf_counter() - t0
     prefix = min(w.N, 4096)
     nh = max(1, min(len(heads_all), int(budget_s / max(one, 1e-3))))
     heads = heads_all[:nh]
     t0 = time.perf_counter()
-    flops = oracle_head_step(x, w, heads, prefix=prefix, dropout=dropout)
+    flops = oracle_head_step(x, w, heads, prefix=prefix, dropout=dropout, fp8=fp8)
     dt = time.perf_counter() - t0
-    sample = (f"oracle fwd{'+bwd' if w.backward else ''} (fp64 NumPy) of {nh} of {len(heads_all)} "
+    bwd = w.backward and not fp8
+    sample = (f"oracle {'fp8 ' if fp8 else ''}fwd{'+bwd' if bwd else ''} (fp64 NumPy) of {nh} of "
+              f"{len(heads_all)} "
               f"heads" + (f", first {prefix} rows/keys of each" if prefix < w.N else "")
               + f"; {dt:.1f} s")
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(),
@@ -239,32 +253,39 @@ def run_reference(args, w, world, rank):
     """The reference arm: the fp64 CPU oracle on bounded samples of the same workload."""
     if rank != 0:
         return 0
-    x = workload_inputs(w)
+    if args.fp8:
+        from exact_io_aware_66_b200.workloads import make_inputs_fp8
+
+        x = make_inputs_fp8(w.B, w.H, w.H, w.N, w.N, w.d, seed=w.seed)
+    else:
+        x = workload_inputs(w)
     steps, warm = args.steps, args.warmup
     budget_per_step = max(0.05, 150.0 / (steps + warm))
     # calibrate a causal-prefix length (multiple of 128) so one step takes about the budget
     t0 = time.perf_counter()
-    oracle_head_step(x, w, [(0, 0)], prefix=min(w.N, 1024))
+    oracle_head_step(x, w, [(0, 0)], prefix=min(w.N, 1024), fp8=args.fp8)
     t1024 = time.perf_counter() - t0
     n = int(min(w.N, 1024 * (budget_per_step / max(t1024, 1e-4)) ** 0.5))
     n = max(128, n // 128 * 128)
     heads = [(0, 0)]
     for _ in range(warm):
-        oracle_head_step(x, w, heads, prefix=n, dropout=args.dropout)
+        oracle_head_step(x, w, heads, prefix=n, dropout=args.dropout, fp8=args.fp8)
     t0 = time.perf_counter()
     flops = 0.0
     for s in range(steps):
         b, h = divmod(s % (w.B * w.H), w.H)
-        flops += oracle_head_step(x, w, [(b, h)], prefix=n, dropout=args.dropout)
+        flops += oracle_head_step(x, w, [(b, h)], prefix=n, dropout=args.dropout, fp8=args.fp8)
     dt = time.perf_counter() - t0
     value = flops / dt / 1e12
-    sample = (f"per step: oracle fwd{'+bwd' if w.backward else ''} (fp64 NumPy) of one head, "
+    bwd = w.backward and not args.fp8
+    sample = (f"per step: oracle {'fp8 ' if args.fp8 else ''}fwd{'+bwd' if bwd else ''} "
+              f"(fp64 NumPy) of one head, "
               f"first {n} of {w.N} rows/keys")
     line = {"impl": "reference", "metric": load_metric(), "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": dt * 1000 / steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1), bf16-rounded, widened to fp64)",
-            "config": workload_config(w, world, args.dropout),
+            "config": workload_config(w, world, args.dropout, args.fp8),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -273,12 +294,14 @@ def run_reference(args, w, world, rank):
     return 0
 
 
-def workload_config(w, world, dropout: float = 0.0) -> dict:
-    return {"workload": w.name + (f"+dropout{dropout:g}" if dropout > 0 else ""),
+def workload_config(w, world, dropout: float = 0.0, fp8: bool = False) -> dict:
+    bwd = w.backward and not fp8
+    return {"workload": w.name + (f"+dropout{dropout:g}" if dropout > 0 else "")
+                        + ("+fp8fwd" if fp8 else ""),
             "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-            "pass": "fwd+bwd" if w.backward else "fwd", "scale": "1/sqrt(d)",
-            "dropout": dropout,
-            "flops_per_step": w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0),
+            "pass": "fwd (E4M3 Q, K, V)" if fp8 else ("fwd+bwd" if bwd else "fwd"),
+            "scale": "1/sqrt(d)", "dropout": dropout,
+            "flops_per_step": w.fwd_flops() + (w.bwd_flops() if bwd else 0.0),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": f"{FLUSH_BYTES >> 20} MiB buffer written before every timed step "
                   f"(L2 is {L2_BYTES >> 20} MiB)"}
@@ -297,11 +320,14 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dropout", type=float, default=0.0)
+    ap.add_argument("--fp8", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if not 0.0 <= args.dropout < 1.0:
         ap.error("--dropout must be in [0, 1)")
+    if args.fp8 and args.dropout > 0:
+        ap.error("--fp8 has no dropout")
     w = WORKLOADS[args.workload]
     world, rank, local = dist_setup()
     if args.impl == "reference":
@@ -311,37 +337,53 @@ def main():
 
     fa.lib()  # fails loudly if the CUDA library is missing: there is no fallback
     dev = torch.device("cuda", local)
-    x = workload_inputs(w)
-    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
-    do = x["do"].to(dev) if w.backward else None
-    o = torch.empty_like(q)
+    backward = w.backward and not args.fp8
+    if args.fp8:
+        from exact_io_aware_66_b200.workloads import make_inputs_fp8
+
+        x = make_inputs_fp8(w.B, w.H, w.H, w.N, w.N, w.d, seed=w.seed)
+        in_names = ("q8", "k8", "v8")
+        q, k, v = (x[n].to(dev) for n in in_names)
+        o = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=dev)
+        ws8 = torch.empty(max(16, fa.fa_fwd_fp8_workspace_size(w.B, w.H, w.H, w.N, w.N, w.d,
+                                                                 w.causal)),
+                          dtype=torch.uint8, device=dev)
+    else:
+        x = workload_inputs(w)
+        in_names = ("q", "k", "v", "do") if backward else ("q", "k", "v")
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        o = torch.empty_like(q)
+    do = x["do"].to(dev) if backward else None
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
-    if w.backward:
+    if backward:
         ws = torch.empty(fa.fa_bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8,
                          device=dev)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     stream = torch.cuda.current_stream(dev)
-
     counter = [0]
 
     def step(q_, k_, v_, do_):
+        if args.fp8:
+            fa.fa_fwd_fp8(q_, k_, v_, x["descale"], o, lse, w.causal, None, stream, ws8)
+            return
         if args.dropout > 0:
             dr = (args.dropout, 0x5EED, counter[0])  # a fresh Philox offset every step
             counter[0] += 1
             fa.fa_fwd_ex(q_, k_, v_, o, lse, w.causal, None, stream, dr)
-            if w.backward:
+            if backward:
                 fa.fa_bwd_ex(q_, k_, v_, o, do_, lse, dq, dk, dv, ws, w.causal, None, stream, dr)
             return
         fa.fa_fwd(q_, k_, v_, o, lse, w.causal, None, stream)
-        if w.backward:
+        if backward:
             fa.fa_bwd(q_, k_, v_, o, do_, lse, dq, dk, dv, ws, w.causal, None, stream)
 
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         step(q, k, v, do)
     fa.fa_check_status(stream)
-    flops_step = workload_config(w, world)["flops_per_step"]
-    launches_per_step = 1 + (3 if w.backward else 0)
+    cfg = workload_config(w, world, args.dropout, args.fp8)
+    flops_step = cfg["flops_per_step"]
+    launches_per_step = (2 if args.fp8 else 1) + (3 if backward else 0)
 
     # ---- timed region: K steps, L2 flushed before each (outside the event pairs) ----
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -370,25 +412,32 @@ def main():
 
     # per-kernel device time from the library's own event pairs
     kern = {name: {"launches": n, "ms": t} for name, (n, t) in prof.items() if n}
-    fwd_ms = kern.get("fa_fwd_kernel", {}).get("ms", 0.0) / args.steps
+    fwd_ms = (kern.get("fa_fwd_kernel", {}).get("ms", 0.0)
+              + kern.get("fa_fwd_fp8_kernel", {}).get("ms", 0.0)
+              + kern.get("fa_fp8_transpose_v", {}).get("ms", 0.0)) / args.steps
     bwd_ms = sum(kern.get(n, {}).get("ms", 0.0)
                  for n in ("fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert")) / args.steps
     peaks = load_peaks()
     dom = max(kern, key=lambda n: kern[n]["ms"])
-    dom_flops = {"fa_fwd_kernel": w.fwd_flops(), "fa_bwd_main": w.bwd_flops()}.get(dom)
+    dom_flops = {"fa_fwd_kernel": w.fwd_flops(), "fa_bwd_main": w.bwd_flops(),
+                 "fa_fwd_fp8_kernel": w.fwd_flops()}.get(dom)
     avg_ms = kern[dom]["ms"] / kern[dom]["launches"]
-    peak = peaks["bf16_sustained"] if ms_total > 1000 else peaks["bf16_burst"]
+    sustained = ms_total > 1000
+    peak = peaks["bf16_sustained"] if sustained else peaks["bf16_burst"]
+    peak_source = (f"{peaks['source']} bf16 {'sustained' if sustained else 'burst'} "
+                   f"(MEASURED_PEAKS.json)")
+    if dom == "fa_fwd_fp8_kernel":  # E4M3 contraction: nominal FP8/bf16 dense ratio 4.5/2.25
+        peak *= 2.0
+        peak_source += " x 2 (nominal fp8/bf16 dense ratio)"
     achieved = dom_flops / (avg_ms / 1e3) / 1e12 if dom_flops else None
     roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak if achieved else None,
-                "traffic": ncu_traffic(dom, workload_config(w, world, args.dropout)["workload"]),
-                "peak_source": f"{peaks['source']} bf16 "
-                               f"{'sustained' if ms_total > 1000 else 'burst'} (MEASURED_PEAKS.json)",
-                "per_launch_flops": dom_flops, "avg_launch_ms": avg_ms}
+                "traffic": ncu_traffic(dom, cfg["workload"]),
+                "peak_source": peak_source, "per_launch_flops": dom_flops, "avg_launch_ms": avg_ms}
 
     # ---- end-to-end: pinned host inputs in, every output back, inside the timed region ----
-    host_in = {n: x[n].pin_memory() for n in (("q", "k", "v", "do") if w.backward else ("q", "k", "v"))}
-    outs = [o, lse] + ([dq, dk, dv] if w.backward else [])
+    host_in = {n: x[n].pin_memory() for n in in_names}
+    outs = [o, lse] + ([dq, dk, dv] if backward else [])
     host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
     dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
@@ -397,7 +446,7 @@ def main():
     def e2e_step():
         for n, t in host_in.items():
             dev_in[n].copy_(t, non_blocking=True)
-        step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in.get("do"))
+        step(*(dev_in[n] for n in in_names[:3]), dev_in.get("do"))
         for t, h in zip(outs, host_out):
             h.copy_(t, non_blocking=True)
 
@@ -420,16 +469,18 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, x, dropout=args.dropout)
+        cpu = cpu_baseline(w, x, dropout=args.dropout, fp8=args.fp8)
 
     if rank == 0:
         line = {
             "metric": load_metric(), "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3" if args.fp8 else "bf16",
             "data": "synthetic (seeded N(0,1)" + (f" x{w.mult}" if w.mult != 1 else "")
-                    + ", bf16), inputs resident in device memory",
-            "config": workload_config(w, world, args.dropout),
+                    + (", E4M3 with per-tensor descale" if args.fp8 else ", bf16")
+                    + "), inputs resident in device memory",
+            "config": cfg,
             "fwd_tflops": w.fwd_flops() / (fwd_ms / 1e3) / 1e12 if fwd_ms else None,
             "bwd_tflops": (w.bwd_flops() / (bwd_ms / 1e3) / 1e12) if bwd_ms else None,
             "frac_of_peak": {"fwd+bwd": value / world / peaks["bf16_burst"],

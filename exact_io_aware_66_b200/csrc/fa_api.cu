@@ -14,6 +14,7 @@
 
 #include "../../include/fa.h"
 #include "fa_bwd.cuh"
+#include "fa_fwd_fp8.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -33,9 +34,11 @@ fa_status cuda_err(cudaError_t e, const char* what) {
 }
 
 // ---- optional per-kernel device timing (fa_profile_enable / fa_profile_read) ----
-constexpr int kKernelKinds = 4;  // fwd, bwd preprocess, bwd main, bwd dQ convert
-const char* const kKernelNames[kKernelKinds] = {"fa_fwd_kernel", "fa_bwd_preprocess",
-                                                "fa_bwd_main", "fa_bwd_dq_convert"};
+// fwd, bwd preprocess, bwd main, bwd dQ convert, fp8 fwd, fp8 V transpose
+constexpr int kKernelKinds = 6;
+const char* const kKernelNames[kKernelKinds] = {"fa_fwd_kernel",     "fa_bwd_preprocess",
+                                                "fa_bwd_main",       "fa_bwd_dq_convert",
+                                                "fa_fwd_fp8_kernel", "fa_fp8_transpose_v"};
 struct ProfileRec {
   int kind;
   cudaEvent_t start, stop;
@@ -83,6 +86,7 @@ struct DeviceState {
   bool checked = false;   // compute capability verified
   bool is_sm100 = false;
   bool fwd_attr[2][2][2] = {};  // [d==128][causal][dropout]: shared-memory attribute set
+  bool fp8_attr[2] = {};        // [causal]
   bool bwd_attr[2][2][2] = {};
 };
 std::mutex g_mu;
@@ -470,6 +474,119 @@ fa_status bwd_checked(const void* q, const void* k, const void* v, const void* o
                       static_cast<cudaStream_t>(stream));
 }
 
+// ---- FP8 forward ----
+size_t fp8_vt_ld(int N_kv) { return (static_cast<size_t>(N_kv) + 15) / 16 * 16; }
+size_t fp8_workspace(const Shape& s) {
+  return static_cast<size_t>(s.B) * s.H_kv * s.d * fp8_vt_ld(s.N_kv);
+}
+
+template <bool CAUSAL>
+fa_status launch_fwd_fp8(DeviceState* ds, const void* q8, const void* k8, const void* v8,
+                         float q_descale, float k_descale, float v_descale, void* o, float* lse,
+                         void* workspace, const Shape& s, cudaStream_t stream) {
+  using L = fa::Fp8Layout;
+  auto kern = fa::fa_fwd_fp8_kernel<CAUSAL>;
+  bool& attr = ds->fp8_attr[CAUSAL];
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncSetAttribute(fp8 fwd smem)");
+    cudaFuncAttributes fattr;  // setmaxnreg split assumes 128 registers per thread at launch
+    e = cudaFuncGetAttributes(&fattr, kern);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncGetAttributes(fp8 fwd)");
+    if (fattr.numRegs != 128)
+      return set_err(FA_ERR_CUDA, "fp8 forward kernel built with %d registers per thread",
+                     fattr.numRegs);
+    attr = true;
+  }
+  const int BH = s.B * s.H, BHkv = s.B * s.H_kv;
+  const int ld = static_cast<int>(fp8_vt_ld(s.N_kv));
+  uint8_t* vt = static_cast<uint8_t*>(workspace);
+  CUtensorMap tq, tk, tvt, to;
+  fa_status st;
+  // E4M3 operands: 128-byte rows (d = 64 is zero-extended by the out-of-bounds fill)
+  if ((st = make_map(&tq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, s.N_q, BH, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+    return st;
+  if ((st = make_map(&tk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, s.N_kv, BHkv, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+    return st;
+  if ((st = make_map(&tvt, vt, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.N_kv, s.d, BHkv, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B, ld)) != FA_OK)
+    return st;
+  if ((st = make_bf16_map(&to, o, s.d, s.N_q, BH, 32)) != FA_OK) return st;
+
+  {
+    const dim3 grid((s.N_kv + 63) / 64, s.d / 64, BHkv);
+    if (grid.z > 65535) return set_err(FA_ERR_UNSUPPORTED, "B*H_kv > 65535 for the fp8 path");
+    ProfileScope prof(5, stream);
+    fa::fa_fp8_transpose_v<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(v8), vt, s.N_kv,
+                                                      s.d, ld);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fp8 V transpose launch");
+
+  fa::Fp8Params p;
+  p.lse = lse;
+  p.status = ds->status;
+  p.N = s.N_q;
+  p.N_kv = s.N_kv;
+  p.BH = BH;
+  p.group = s.H / s.H_kv;
+  p.off = s.off();
+  p.n_qblocks = (s.N_q + 255) / 256;
+  p.o_boxes = (s.d + 63) / 64;
+  p.scale_log2 = s.scale * 1.4426950408889634f * q_descale * k_descale;
+  p.o_scale = v_descale;
+  const long long grid = 1LL * p.n_qblocks * BH;
+  if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  {
+    ProfileScope prof(4, stream);
+    kern<<<static_cast<unsigned>(grid), fa::kFwdThreads, L::kAlloc, stream>>>(tq, tk, tvt, to, p);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fp8 forward launch");
+  return FA_OK;
+}
+
+fa_status fp8_checked(const void* q8, const void* k8, const void* v8, float qd, float kd,
+                      float vd, void* o, float* lse, const Shape& s, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  fa_status st = check_shape(s);
+  if (st != FA_OK) return st;
+  if (!q8 || !k8 || !v8 || !o || !lse) return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
+  for (float x : {qd, kd, vd})
+    if (!std::isfinite(x) || !(x > 0.f))
+      return set_err(FA_ERR_INVALID_ARG, "descale factors must be finite and > 0");
+  const void* ptrs[6] = {q8, k8, v8, o, lse, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return set_err(FA_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  const size_t need = fp8_workspace(s);
+  if (!workspace || workspace_bytes < need)
+    return set_err(FA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
+                   need);
+  const size_t qb = static_cast<size_t>(s.B) * s.H * s.N_q * s.d;
+  const size_t kvb = static_cast<size_t>(s.B) * s.H_kv * s.N_kv * s.d;
+  const void* ins[3] = {q8, k8, v8};
+  const size_t insz[3] = {qb, kvb, kvb};
+  void* outs[3] = {o, lse, workspace};
+  const size_t outsz[3] = {s.q_bytes(), s.lse_bytes(), need};
+  for (int a = 0; a < 3; ++a) {
+    for (int b = 0; b < 3; ++b)
+      if (overlaps(outs[a], outsz[a], ins[b], insz[b]))
+        return set_err(FA_ERR_INVALID_ARG, "outputs/workspace must not alias inputs");
+    for (int b = a + 1; b < 3; ++b)
+      if (overlaps(outs[a], outsz[a], outs[b], outsz[b]))
+        return set_err(FA_ERR_INVALID_ARG, "outputs/workspace must not overlap each other");
+  }
+  DeviceState* ds = device_state(&st);
+  if (!ds) return st;
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return s.mask != 0
+             ? launch_fwd_fp8<true>(ds, q8, k8, v8, qd, kd, vd, o, lse, workspace, s, cs)
+             : launch_fwd_fp8<false>(ds, q8, k8, v8, qd, kd, vd, o, lse, workspace, s, cs);
+}
+
 Shape from_public(const fa_attn_shape* p) {
   return Shape{p->B, p->H, p->H_kv, p->N_q, p->N_kv, p->d, p->scale, p->mask};
 }
@@ -563,6 +680,25 @@ fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, 
   const fa_status st = apply_dropout(s, dropout);
   if (st != FA_OK) return st;
   return bwd_checked(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, s, stream);
+}
+
+size_t fa_fwd_fp8_workspace_size(const fa_attn_shape* shape) {
+  if (!shape) return 0;
+  const Shape s = from_public(shape);
+  const char saved = g_err[0];
+  const bool ok = check_shape(s) == FA_OK;
+  if (saved == '\0') g_err[0] = '\0';
+  return ok ? fp8_workspace(s) : 0;
+}
+
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_descale,
+                     float k_descale, float v_descale, void* o, float* lse,
+                     const fa_attn_shape* shape, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  g_err[0] = '\0';
+  if (!shape) return set_err(FA_ERR_INVALID_ARG, "null shape");
+  return fp8_checked(q8, k8, v8, q_descale, k_descale, v_descale, o, lse, from_public(shape),
+                     workspace, workspace_bytes, stream);
 }
 
 fa_status fa_profile_enable(int on) {

@@ -41,6 +41,8 @@ SIGNATURES = {
     "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "fa_bwd_ex_workspace_size": (_Z, [_P]),
     "fa_bwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P, _P]),
+    "fa_fwd_fp8_workspace_size": (_Z, [_P]),
+    "fa_fwd_fp8": (_I, [_P, _P, _P, _F, _F, _F, _P, _P, _P, _P, _Z, _P]),
 }
 
 # fa_mask values
@@ -80,7 +82,7 @@ def mask_code(causal) -> int:
     raise ValueError(f"unknown mask {causal!r}")
 
 
-KERNEL_KINDS = 4
+KERNEL_KINDS = 6
 
 _lib = None
 
@@ -282,6 +284,55 @@ def fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, causal=False,
     wbytes = workspace.numel() * workspace.element_size()
     _check("fa_bwd_ex", lib().fa_bwd_ex(*ptrs, workspace.data_ptr(), wbytes, ctypes.byref(s),
                                         _dropout_arg(dropout), _stream_handle(stream)))
+
+
+def _req8(x: torch.Tensor, name: str):
+    if not isinstance(x, torch.Tensor) or not x.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if x.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise ValueError(f"{name} must hold E4M3 codes (torch.float8_e4m3fn or uint8)")
+    if not x.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return x.data_ptr()
+
+
+def fa_fwd_fp8_workspace_size(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int,
+                              causal=False) -> int:
+    s = FaAttnShape(B, H, H_kv, N_q, N_kv, d, default_scale(d) if d > 0 else 1.0,
+                    mask_code(causal))
+    return int(lib().fa_fwd_fp8_workspace_size(ctypes.byref(s)))
+
+
+def fa_fwd_fp8(q8, k8, v8, descale, o, lse, causal=False, scale: float | None = None,
+               stream=None, workspace=None):
+    """FP8 forward: q8 [B,H,N_q,d], k8 and v8 [B,H_kv,N_kv,d] E4M3 codes with descale =
+    (q, k, v) fp32 factors, into caller-allocated o (bf16, like q8) and lse (fp32 [B,H,N_q]).
+    Allocates the V^T workspace unless one is given."""
+    s = _shape(q8, k8, v8, causal, scale)
+    if _dims(o) != (s.B, s.H, s.N_q, s.d):
+        raise ValueError("o shape mismatch")
+    if tuple(lse.shape) != (s.B, s.H, s.N_q):
+        raise ValueError("lse must be [B, H, N_q]")
+    if workspace is None:
+        workspace = torch.empty(max(16, int(lib().fa_fwd_fp8_workspace_size(ctypes.byref(s)))),
+                                dtype=torch.uint8, device=q8.device)
+    qd, kd, vd = (float(x) for x in descale)
+    ptrs = [_req8(q8, "q8"), _req8(k8, "k8"), _req8(v8, "v8")]
+    _check("fa_fwd_fp8", lib().fa_fwd_fp8(*ptrs, qd, kd, vd, _req(o, "o"),
+                                          _req(lse, "lse", torch.float32), ctypes.byref(s),
+                                          workspace.data_ptr(),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream_handle(stream)))
+
+
+def attention_forward_fp8(q8, k8, v8, descale, causal=False, scale: float | None = None,
+                          stream=None):
+    """Returns (o bf16, lse fp32) of the FP8 forward (see fa_fwd_fp8)."""
+    B, H, N, d = _dims(q8)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    fa_fwd_fp8(q8, k8, v8, descale, o, lse, causal, scale, stream)
+    return o, lse
 
 
 def attention_forward(q, k, v, causal=False, scale: float | None = None, stream=None,

@@ -97,6 +97,23 @@ def make_inputs_ex(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int, seed:
     return out
 
 
+def make_inputs_fp8(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int, seed: int) -> dict:
+    """E4M3 inputs: {'q8','k8','v8'} as contiguous torch.float8_e4m3fn CPU tensors (q8 of shape
+    [B, H, N_q, d], k8 and v8 of shape [B, H_kv, N_kv, d]) and {'descale': (q, k, v)}, fp32
+    factors. Standard normal draws, each tensor divided by amax / 448 and rounded to E4M3 by
+    torch, so the codes span E4M3's range; the value of a code is its E4M3 value times its
+    factor."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    out, descale = {}, []
+    for name, (h, n) in (("q8", (H, N_q)), ("k8", (H_kv, N_kv)), ("v8", (H_kv, N_kv))):
+        x = torch.randn(B, h, n, d, dtype=torch.float32, generator=g)
+        f = float(torch.tensor(float(x.abs().max()) / 448.0, dtype=torch.float32))
+        out[name] = (x / f).to(torch.float8_e4m3fn).contiguous()
+        descale.append(f)
+    out["descale"] = tuple(descale)
+    return out
+
+
 def workload_inputs(w: Workload, with_do: bool | None = None) -> dict:
     if with_do is None:
         with_do = w.backward

@@ -155,15 +155,35 @@ fa_status fa_selftest_timeout(int limit_us, void* stream);
  * Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA. */
 fa_status fa_check_status(void* stream);
 
+/* FP8 forward: q8, k8, v8 hold E4M3 codes (OCP 8-bit floating point, the "e4m3fn" encoding:
+ * bias 7, no infinities, largest finite 448) in the layouts of fa_attn_shape, one byte per
+ * element; the value of each element is its E4M3 value times the tensor's descale factor
+ * (finite, > 0). Computes the same O (bf16) and lse (fp32) as fa_fwd_ex on those values, with
+ * both products on 8-bit tensor cores: S = Q K^T accumulates exact E4M3 products in fp32, and
+ * the probabilities are rounded to E4M3 for the product with V (O is normalised by the sum of
+ * the rounded weights; lse uses the unrounded sum). The pages name FP8 only as a feature of a
+ * later FlashAttention version ("How does FlashAttention optimize memory and speed via
+ * tiling?", "Interview tips"); this entry point is that reading of it. Forward only; no
+ * dropout; d in {64, 128}; B * H_kv <= 65535. The workspace (caller-owned, at least
+ * fa_fwd_fp8_workspace_size bytes, 16-byte aligned; 0 for an invalid shape) receives V
+ * transposed to [B, H_kv, d, N_kv rounded up to 16]. Errors as fa_fwd_ex, and
+ * FA_ERR_WORKSPACE for a missing or short workspace. */
+size_t fa_fwd_fp8_workspace_size(const fa_attn_shape* shape);
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_descale,
+                     float k_descale, float v_descale, void* o, float* lse,
+                     const fa_attn_shape* shape, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
 /* Optional device-side timing of the library's own kernels, for benchmarks and tracing.
- * While enabled on the calling thread, every kernel fa_fwd / fa_bwd launches is bracketed by a
+ * While enabled on the calling thread, every kernel the library launches is bracketed by a
  * pair of CUDA events recorded on its launch stream. fa_profile_read() waits for those events
  * and writes, per kernel kind k (0 = forward, 1 = backward preprocess, 2 = backward main,
- * 3 = backward dQ conversion; FA_KERNEL_KINDS in total), the number of launches to
+ * 3 = backward dQ conversion, 4 = FP8 forward, 5 = FP8 V transpose; FA_KERNEL_KINDS in
+ * total), the number of launches to
  * launches[k] and their summed device time in milliseconds to ms[k], then forgets them.
  * n is the length of both arrays (>= FA_KERNEL_KINDS). Events are created by the library and
  * reused; no device memory is allocated. */
-#define FA_KERNEL_KINDS 4
+#define FA_KERNEL_KINDS 6
 fa_status fa_profile_enable(int on);
 fa_status fa_profile_read(double* ms, long long* launches, int n);
 /* Name of kernel kind k ("" if out of range). */
