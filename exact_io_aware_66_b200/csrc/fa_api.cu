@@ -208,8 +208,8 @@ fa_status check_shape(const Shape& s) {
                    s.B, s.H, s.H_kv, s.N_q, s.N_kv);
   if (s.H % s.H_kv != 0)
     return set_err(FA_ERR_INVALID_ARG, "H=%d is not a multiple of H_kv=%d", s.H, s.H_kv);
-  if (s.d != 64 && s.d != 128)
-    return set_err(FA_ERR_UNSUPPORTED, "head dim d=%d not in {64, 128}", s.d);
+  if (s.d != 64 && s.d != 96 && s.d != 128)
+    return set_err(FA_ERR_UNSUPPORTED, "head dim d=%d not in {64, 96, 128}", s.d);
   if (s.mask < 0 || s.mask > 2) return set_err(FA_ERR_INVALID_ARG, "mask mode %d unknown", s.mask);
   const long long rows_q = 1LL * s.B * s.H * s.N_q, rows_kv = 1LL * s.B * s.H_kv * s.N_kv;
   if (rows_q >= (1LL << 31) || rows_kv >= (1LL << 31))
@@ -259,10 +259,12 @@ fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* 
   const int BH = s.B * s.H, BHkv = s.B * s.H_kv;
   CUtensorMap tq, tk, tv, to;
   fa_status st;
-  if ((st = make_bf16_map(&tq, q, D, s.N_q, BH, 128)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tk, k, D, s.N_kv, BHkv, 128)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tv, v, D, s.N_kv, BHkv, 128)) != FA_OK) return st;
-  if ((st = make_bf16_map(&to, o, D, s.N_q, BH, 32)) != FA_OK) return st;
+  // global width s.d (96 runs the D = 128 kernel: the loads zero-fill columns 96..127, the
+  // stores clip them)
+  if ((st = make_bf16_map(&tq, q, s.d, s.N_q, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tk, k, s.d, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tv, v, s.d, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&to, o, s.d, s.N_q, BH, 32)) != FA_OK) return st;
   fa::FwdParams p;
   p.lse = lse;
   p.status = ds->status;
@@ -300,19 +302,19 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   const int BH = s.B * s.H, BHkv = s.B * s.H_kv, N = s.N_q;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(ws);
-  float* Dvec = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_D(BH, N, D));
-  float* lse2 = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_lse2(BH, N, D));
+  float* Dvec = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_D(BH, N, s.d));
+  float* lse2 = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_lse2(BH, N, s.d));
   const int n64 = static_cast<int>(fa::bwd_n64(N));
   const long long rows = 1LL * BH * N;
 
   CUtensorMap tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv;
   fa_status st;
-  if ((st = make_bf16_map(&tq, q, D, N, BH, 64)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tk, k, D, s.N_kv, BHkv, 128)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tv, v, D, s.N_kv, BHkv, 128)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tdo, dO, D, N, BH, 64)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tdk, dk, D, s.N_kv, BHkv, 32)) != FA_OK) return st;
-  if ((st = make_bf16_map(&tdv, dv, D, s.N_kv, BHkv, 32)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tq, q, s.d, N, BH, 64)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tk, k, s.d, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tv, v, s.d, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdo, dO, s.d, N, BH, 64)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdk, dk, s.d, s.N_kv, BHkv, 32)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdv, dv, s.d, s.N_kv, BHkv, 32)) != FA_OK) return st;
   // per-row fp32 vectors: [BH][N_q] with a row stride of N64 elements, 64-element boxes
   if ((st = make_map(&tl, lse2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 64, 1,
                      CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
@@ -320,20 +322,25 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   if ((st = make_map(&tD, Dvec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 64, 1,
                      CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
     return st;
-  // dQ accumulator: fp32 [BH][N_q][D], reduction boxes of 32 columns x 64 rows
-  if ((st = make_map(&tacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, N, BH, 32, 64,
+  // dQ accumulator: fp32 [BH][N_q][d], reduction boxes of 32 columns x 64 rows
+  if ((st = make_map(&tacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, s.d, N, BH, 32, 64,
                      CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
     return st;
 
-  constexpr int tpr = D / 8;
-  const long long prep_threads = rows * tpr;
+  const long long prep_threads = rows * (s.d <= 64 ? 8 : 16);
   const long long prep_blocks = (prep_threads + fa::kPrepThreads - 1) / fa::kPrepThreads;
   if (prep_blocks >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
   {
     ProfileScope prof(1, stream);
-    fa::fa_bwd_preprocess<D><<<static_cast<unsigned>(prep_blocks), fa::kPrepThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dq_acc,
-        Dvec, lse2, rows, N, n64);
+    const auto* o16 = static_cast<const __nv_bfloat16*>(o);
+    const auto* do16 = static_cast<const __nv_bfloat16*>(dO);
+    const unsigned nb = static_cast<unsigned>(prep_blocks);
+    if (s.d == 96)
+      fa::fa_bwd_preprocess<96><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc, Dvec,
+                                                                     lse2, rows, N, n64);
+    else
+      fa::fa_bwd_preprocess<D><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc, Dvec,
+                                                                    lse2, rows, N, n64);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd preprocess launch");
@@ -347,6 +354,7 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   p.off = s.off();
   p.n_kv = (s.N_kv + 127) / 128;
   p.n_q = (N + 63) / 64;
+  p.d = s.d;
   {
     // key/value heads per scheduling group: a group's K, V, and its query heads' Q, dO (bf16)
     // and fp32 dQ accumulator should stay within about half of the 126 MB L2
@@ -368,7 +376,7 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd main launch");
 
-  const long long n8 = rows * D / 8;
+  const long long n8 = rows * s.d / 8;
   {
     ProfileScope prof(3, stream);
     fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
@@ -517,7 +525,7 @@ fa_status launch_fwd_fp8(DeviceState* ds, const void* q8, const void* k8, const 
   if ((st = make_bf16_map(&to, o, s.d, s.N_q, BH, 32)) != FA_OK) return st;
 
   {
-    const dim3 grid((s.N_kv + 63) / 64, s.d / 64, BHkv);
+    const dim3 grid((s.N_kv + 63) / 64, (s.d + 63) / 64, BHkv);
     if (grid.z > 65535) return set_err(FA_ERR_UNSUPPORTED, "B*H_kv > 65535 for the fp8 path");
     ProfileScope prof(5, stream);
     fa::fa_fp8_transpose_v<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(v8), vt, s.N_kv,
@@ -648,7 +656,7 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 96 && d != 128)) return 0;
   return fa::bwd_workspace_bytes(static_cast<size_t>(B) * H, N, d);
 }
 

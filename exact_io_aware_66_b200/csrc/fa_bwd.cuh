@@ -47,7 +47,8 @@ inline size_t bwd_workspace_bytes(size_t BH, int N, int d) {
 }
 
 // ------------------------------------------------------------------------------------------
-// 1. Preprocess: one group of d/8 threads per row; each thread owns 8 columns.
+// 1. Preprocess: one group of TPR threads per row (d/8 rounded up to a power of two); each
+//    thread owns 8 columns (threads past the row's d/8 chunks only join the reduction).
 // ------------------------------------------------------------------------------------------
 constexpr int kPrepThreads = 256;
 
@@ -57,12 +58,13 @@ __global__ void __launch_bounds__(kPrepThreads)
                       const float* __restrict__ lse, float* __restrict__ dq_acc,
                       float* __restrict__ Dvec, float* __restrict__ lse2, long long rows, int N,
                       int n64) {
-  constexpr int TPR = D / 8;  // threads per row
+  constexpr int TPR = D <= 64 ? 8 : 16;  // threads per row
+  static_assert(D % 8 == 0 && D / 8 <= TPR, "preprocess row split");
   const long long t = static_cast<long long>(blockIdx.x) * kPrepThreads + threadIdx.x;
   const long long row = t / TPR;
   const int part = static_cast<int>(t % TPR);
   float acc = 0.f;
-  if (row < rows) {
+  if (row < rows && part * 8 < D) {
     const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
     const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
     const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
@@ -160,6 +162,7 @@ struct BwdParams {
   int n_kv;        // ceil(N_kv / 128)
   int n_q;         // ceil(N / 64)
   int group;       // key/value heads per scheduling group
+  int d;           // head dimension of the tensors (<= D; columns past d are zero-filled)
   float scale;
   float scale_log2;
   DropoutParams drop;  // read only by the DROPOUT instantiations
@@ -398,7 +401,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     float* stagef = reinterpret_cast<float*>(gbase + L::kDQ + wq * 8192);
     const uint32_t stage_s = sbase + L::kDQ + wq * 8192;
-    const bool active = 32 * wq < D;
+    const bool active = 32 * wq < p.d;
     bool ok = true;
     for (int i = 0; i < n_i; ++i) {
       const int b = i & 1;

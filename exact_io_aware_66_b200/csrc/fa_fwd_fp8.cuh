@@ -9,9 +9,9 @@
 // probabilities P are rounded to E4M3 for the PV product, and O is normalised by the sum of
 // exactly those rounded weights. O is written in bf16, lse in fp32 from the unrounded sum.
 //
-// Layout: one internal head dimension of 128 bytes per row (d = 64 is zero-extended by the TMA
-// loads). The PV product wants V with the key index contiguous (K-major B operand), so V is
-// first transposed into a workspace [B*H_kv][d][N_kv padded to 16] by fa_fp8_transpose_v.
+// Layout: one internal head dimension of 128 bytes per row (d = 64 or 96 is zero-extended by
+// the TMA loads). The PV product wants V with the key index contiguous (K-major B operand), so
+// V is first transposed into a workspace [B*H_kv][d][N_kv padded to 16] by fa_fp8_transpose_v.
 //
 // Roles (16 warps), TMEM and the issue order are those of fa_fwd.cuh; P takes 32 TMEM columns
 // (four E4M3 per column) at the start of its S buffer.
@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 }
 
 // V [rows][d] (E4M3 bytes) -> V^T [d][ld] per head, 64 x 64-byte tiles through shared memory.
-// Grid: (ceil(N_kv / 64), d / 64, B * H_kv), 256 threads.
+// Grid: (ceil(N_kv / 64), ceil(d / 64), B * H_kv), 256 threads; d a multiple of 16.
 __global__ void __launch_bounds__(256)
     fa_fp8_transpose_v(const uint8_t* __restrict__ v, uint8_t* __restrict__ vt, int N_kv, int d,
                        int ld) {
@@ -446,14 +446,14 @@ __global__ void __launch_bounds__(256)
   const int r = threadIdx.x >> 2, part = (threadIdx.x & 3) * 16;
   {
     uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (k0 + r < N_kv)
+    if (k0 + r < N_kv && c0 + part < d)  // d is a multiple of 16
       x = *reinterpret_cast<const uint4*>(v + (head * N_kv + k0 + r) * d + c0 + part);
     const uint8_t* b = reinterpret_cast<const uint8_t*>(&x);
 #pragma unroll
     for (int i = 0; i < 16; ++i) tile[r][part + i] = b[i];
   }
   __syncthreads();
-  if (k0 + part < N_kv) {  // chunk of 16 keys starting inside the row (ld is a multiple of 16)
+  if (k0 + part < N_kv && c0 + r < d) {  // 16 keys starting inside the row (ld % 16 == 0)
     uint4 y;
     uint8_t* b = reinterpret_cast<uint8_t*>(&y);
 #pragma unroll

@@ -51,7 +51,8 @@ typedef enum {
   FA_ERR_WORKSPACE = 6    /* backward workspace missing or smaller than fa_bwd_workspace_size */
 } fa_status;
 
-/* Limits: d in {64, 128}; B, H, N >= 1; B*H*N < 2^31; B*H*ceil(N/256) < 2^31. */
+/* Limits: d in {64, 96, 128} (96 runs the d = 128 kernels on zero-filled columns); B, H, N >= 1;
+ * B*H*N < 2^31; B*H*ceil(N/256) < 2^31. */
 
 /* Masks of the extended entry points. */
 typedef enum {
@@ -66,7 +67,7 @@ typedef enum {
  * uses key/value head h / (H / H_kv) (grouped heads; H_kv = 1 is a single shared K/V head),
  * and dk, dv of a key/value head sum over the query heads that share it. A query row that sees
  * no key (FA_MASK_CAUSAL_BOTTOM_RIGHT with N_q > N_kv) gets o = 0, lse = -inf and dq = 0.
- * Limits: d in {64, 128}; all sizes >= 1; B*H*N_q and B*H_kv*N_kv < 2^31. */
+ * Limits: d in {64, 96, 128}; all sizes >= 1; B*H*N_q and B*H_kv*N_kv < 2^31. */
 typedef struct {
   int B, H, H_kv, N_q, N_kv, d;
   float scale; /* finite, > 0; normally 1/sqrt(d) */
@@ -164,7 +165,7 @@ fa_status fa_check_status(void* stream);
  * the rounded weights; lse uses the unrounded sum). The pages name FP8 only as a feature of a
  * later FlashAttention version ("How does FlashAttention optimize memory and speed via
  * tiling?", "Interview tips"); this entry point is that reading of it. Forward only; no
- * dropout; d in {64, 128}; B * H_kv <= 65535. The workspace (caller-owned, at least
+ * dropout; d in {64, 96, 128}; B * H_kv <= 65535. The workspace (caller-owned, at least
  * fa_fwd_fp8_workspace_size bytes, 16-byte aligned; 0 for an invalid shape) receives V
  * transposed to [B, H_kv, d, N_kv rounded up to 16]. Errors as fa_fwd_ex, and
  * FA_ERR_WORKSPACE for a missing or short workspace. */

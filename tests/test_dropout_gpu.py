@@ -90,6 +90,7 @@ CASES = [  # (B, H, H_kv, N_q, N_kv, d, mask, p)
     (1, 2, 2, 100, 700, 128, "bottom_right", 0.5),
     (1, 4, 1, 513, 513, 64, True, 0.17),
     (1, 2, 1, 640, 130, 128, False, 0.9),
+    (1, 2, 2, 300, 300, 96, True, 0.2),
 ]
 
 

@@ -33,6 +33,9 @@ CASES = [  # (B, H, H_kv, N_q, N_kv, d, mask)
     (1, 2, 2, 600, 200, 128, True),
     (1, 3, 1, 130, 900, 128, False),
     (1, 2, 2, 384, 128, 64, False),
+    (1, 2, 2, 300, 300, 96, False),             # d = 96: the d = 128 kernels, zero-filled
+    (2, 4, 2, 513, 513, 96, True),
+    (1, 2, 1, 100, 700, 96, "bottom_right"),
 ]
 
 

@@ -95,6 +95,7 @@ CASES = [  # (B, H, H_kv, N_q, N_kv, d, mask)
     (1, 2, 2, 100, 700, 128, "bottom_right"),
     (1, 2, 2, 700, 300, 64, "bottom_right"),
     (1, 2, 1, 1000, 1000, 64, False),
+    (1, 2, 2, 333, 333, 96, True),
 ]
 
 
