@@ -22,3 +22,4 @@ from .attention import (  # noqa: F401
     tiled_attention_forward,
 )
 from .dropout import dropout_keep, dropout_p8, keep_scale, philox4x32_10  # noqa: F401
+from .fp8 import attention_forward_fp8, e4m3_decode  # noqa: F401
