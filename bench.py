@@ -26,6 +26,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -68,11 +69,20 @@ def load_peaks() -> dict:
                 "source": "fallback"}
 
 
+def _code_only(src: str) -> str:
+    """The source without comments and blank lines: what the compiler sees."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def sources_hash() -> str:
+    """Fingerprint of the kernel and host sources (comments excluded), recorded with each ncu
+    capture so that bench.py reports its traffic only while the code is unchanged."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

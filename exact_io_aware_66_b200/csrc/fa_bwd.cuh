@@ -10,9 +10,10 @@
 //
 // Three kernels run in order on the caller's stream:
 //   1. fa_bwd_preprocess: D = rowsum(dO o O) (fp32), lse2 = -lse * log2(e), dQ_acc = 0.
-//   2. fa_bwd_main: one CTA per (head, 128-key tile j). K_j and V_j stay in shared memory;
-//      64-row tiles of Q and dO stream through a 2-stage TMA ring. Per query tile i, five
-//      tcgen05 MMAs (all M = 128):
+//   2. fa_bwd_main: one CTA per (key/value head, 128-key tile j), looping over every query
+//      head that shares the key/value head and over the 64-row query tiles that see tile j.
+//      K_j and V_j stay in shared memory; tiles of Q and dO stream through a 3-stage TMA ring
+//      (4 at d = 64). Per query tile i, five tcgen05 MMAs (all M = 128):
 //          S^T  = K_j Q_i^T          -> TMEM (64 columns, double buffered)
 //          dP^T = V_j dO_i^T         -> TMEM (64 columns, double buffered)
 //          dV  += P^T dO_i           (A = P^T from TMEM, bf16)            -> TMEM, d columns
@@ -21,7 +22,9 @@
 //      Two warpgroups turn S^T/dP^T into P^T (back to TMEM) and dS^T (to shared memory) while
 //      the tensor core works on the previous tile; a third drains dQ^T from TMEM and adds it
 //      into the fp32 accumulator with TMA bulk reductions (cp.reduce.async.bulk .add.f32).
-//      The final dK (times scale) and dV are stored with TMA.
+//      The final dK (times scale) and dV are stored with TMA. With dropout (DROPOUT), the
+//      elementwise warps regenerate the keep decisions of the forward (dropout.cuh) and form
+//      dS = P o (r Z o dP - D) and Z o P for the dV product; dV is scaled by r at the end.
 //   3. fa_bwd_dq_convert: dQ = bf16(dQ_acc).
 #pragma once
 #include "dropout.cuh"

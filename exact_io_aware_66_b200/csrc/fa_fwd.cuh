@@ -21,6 +21,9 @@
 // straight from TMEM, so P never touches shared memory.
 // MMA issue order per key tile j: PV0(j), S0(j+1), PV1(j), S1(j+1) — while softmax 0 works on
 // S0(j+1) the tensor core runs PV1(j) and S1(j+1), and vice versa.
+// Variants: grouped K/V heads (query head h reads K/V head h / group), a causal offset for
+// unequal lengths (key j visible to query i iff j <= i + off), and dropout on P (DROPOUT; keep
+// decisions from dropout.cuh).
 #pragma once
 #include "dropout.cuh"
 #include "sm100.cuh"
