@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -85,9 +86,11 @@ struct DeviceState {
   int* status = nullptr;  // device status word
   bool checked = false;   // compute capability verified
   bool is_sm100 = false;
-  bool fwd_attr[2][2][2] = {};  // [d==128][causal][dropout]: shared-memory attribute set
-  bool fp8_attr[2] = {};        // [causal]
-  bool bwd_attr[2][2][2] = {};
+  // cudaFuncSetAttribute done for [d == 128][causal][dropout] (atomic: calls from several host
+  // threads may launch concurrently; setting an attribute twice is harmless)
+  std::atomic<bool> fwd_attr[2][2][2] = {};
+  std::atomic<bool> fp8_attr[2] = {};  // [causal]
+  std::atomic<bool> bwd_attr[2][2][2] = {};
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -241,7 +244,7 @@ fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* 
                      float* lse, const Shape& s, cudaStream_t stream) {
   using L = fa::FwdLayout<D>;
   auto kern = fa::fa_fwd_kernel<D, CAUSAL, DROPOUT>;
-  bool& attr = ds->fwd_attr[D == 128][CAUSAL][DROPOUT];
+  std::atomic<bool>& attr = ds->fwd_attr[D == 128][CAUSAL][DROPOUT];
   if (!attr) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -292,7 +295,7 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
                      void* workspace, const Shape& s, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
   auto kern = fa::fa_bwd_main<D, CAUSAL, DROPOUT>;
-  bool& attr = ds->bwd_attr[D == 128][CAUSAL][DROPOUT];
+  std::atomic<bool>& attr = ds->bwd_attr[D == 128][CAUSAL][DROPOUT];
   if (!attr) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -494,7 +497,7 @@ fa_status launch_fwd_fp8(DeviceState* ds, const void* q8, const void* k8, const 
                          void* workspace, const Shape& s, cudaStream_t stream) {
   using L = fa::Fp8Layout;
   auto kern = fa::fa_fwd_fp8_kernel<CAUSAL>;
-  bool& attr = ds->fp8_attr[CAUSAL];
+  std::atomic<bool>& attr = ds->fp8_attr[CAUSAL];
   if (!attr) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -629,6 +632,17 @@ struct NoAllocDevice {
   int* status = nullptr;    // device address of g_noalloc_status on this device
   bool bwd_attr[2][2][2] = {};
 };
+
+void copy_flags(std::atomic<bool> (&dst)[2][2][2], const bool (&src)[2][2][2]) {
+  for (int a = 0; a < 2; ++a)
+    for (int b = 0; b < 2; ++b)
+      for (int c = 0; c < 2; ++c) dst[a][b][c].store(src[a][b][c]);
+}
+void copy_flags(bool (&dst)[2][2][2], const std::atomic<bool> (&src)[2][2][2]) {
+  for (int a = 0; a < 2; ++a)
+    for (int b = 0; b < 2; ++b)
+      for (int c = 0; c < 2; ++c) dst[a][b][c] = src[a][b][c].load();
+}
 NoAllocDevice g_noalloc[kMaxDevices];
 
 }  // namespace
@@ -802,7 +816,7 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
     }
     local.status = nd.status;
     local.checked = local.is_sm100 = true;
-    std::memcpy(local.bwd_attr, nd.bwd_attr, sizeof(local.bwd_attr));
+    copy_flags(local.bwd_attr, nd.bwd_attr);
   }
   // The first kernel of the backward rewrites every scratch byte the later ones read (dQ
   // accumulator zeroed, D and -lse*log2e recomputed), so the previous call's contents do not
@@ -811,7 +825,7 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                     static_cast<cudaStream_t>(stream));
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    std::memcpy(g_noalloc[dev].bwd_attr, local.bwd_attr, sizeof(local.bwd_attr));
+    copy_flags(g_noalloc[dev].bwd_attr, local.bwd_attr);
   }
   return st;
 }
