@@ -343,6 +343,10 @@ def main():
     world, rank, local = dist_setup()
     if args.impl == "reference":
         return run_reference(args, w, world, rank)
+    if world > 1:  # each replica computes its own units: inputs seeded per rank
+        import dataclasses
+
+        w = dataclasses.replace(w, seed=w.seed + 7919 * rank)
 
     from exact_io_aware_66_b200 import fa
 
