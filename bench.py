@@ -43,6 +43,7 @@ DEFAULT_WORKLOAD = "causal_train_b4h16n4096d128"
 L2_BYTES = 126 * 1024 * 1024
 FLUSH_BYTES = 512 * 1024 * 1024
 KERNEL_SOURCES = ["exact_io_aware_66_b200/csrc/fa_bwd.cuh", "exact_io_aware_66_b200/csrc/fa_fwd.cuh",
+                  "exact_io_aware_66_b200/csrc/fa_fwd_d256.cuh",
                   "exact_io_aware_66_b200/csrc/sm100.cuh", "exact_io_aware_66_b200/csrc/fa_api.cu",
                   "exact_io_aware_66_b200/csrc/dropout.cuh",
                   "exact_io_aware_66_b200/csrc/fa_fwd_fp8.cuh"]
@@ -427,15 +428,15 @@ def main():
 
     # per-kernel device time from the library's own event pairs
     kern = {name: {"launches": n, "ms": t} for name, (n, t) in prof.items() if n}
-    fwd_ms = (kern.get("fa_fwd_kernel", {}).get("ms", 0.0)
-              + kern.get("fa_fwd_fp8_kernel", {}).get("ms", 0.0)
-              + kern.get("fa_fp8_transpose_v", {}).get("ms", 0.0)) / args.steps
+    fwd_ms = sum(kern.get(n, {}).get("ms", 0.0)
+                 for n in ("fa_fwd_kernel", "fa_fwd_d256_kernel", "fa_fwd_fp8_kernel",
+                           "fa_fp8_transpose_v")) / args.steps
     bwd_ms = sum(kern.get(n, {}).get("ms", 0.0)
                  for n in ("fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert")) / args.steps
     peaks = load_peaks()
     dom = max(kern, key=lambda n: kern[n]["ms"])
     dom_flops = {"fa_fwd_kernel": w.fwd_flops(), "fa_bwd_main": w.bwd_flops(),
-                 "fa_fwd_fp8_kernel": w.fwd_flops()}.get(dom)
+                 "fa_fwd_fp8_kernel": w.fwd_flops(), "fa_fwd_d256_kernel": w.fwd_flops()}.get(dom)
     avg_ms = kern[dom]["ms"] / kern[dom]["launches"]
     sustained = ms_total > 1000
     peak = peaks["bf16_sustained"] if sustained else peaks["bf16_burst"]

@@ -15,6 +15,7 @@
 
 #include "../../include/fa.h"
 #include "fa_bwd.cuh"
+#include "fa_fwd_d256.cuh"
 #include "fa_fwd_fp8.cuh"
 #include "fa_fwd.cuh"
 
@@ -35,11 +36,11 @@ fa_status cuda_err(cudaError_t e, const char* what) {
 }
 
 // ---- optional per-kernel device timing (fa_profile_enable / fa_profile_read) ----
-// fwd, bwd preprocess, bwd main, bwd dQ convert, fp8 fwd, fp8 V transpose
-constexpr int kKernelKinds = 6;
-const char* const kKernelNames[kKernelKinds] = {"fa_fwd_kernel",     "fa_bwd_preprocess",
-                                                "fa_bwd_main",       "fa_bwd_dq_convert",
-                                                "fa_fwd_fp8_kernel", "fa_fp8_transpose_v"};
+// fwd, bwd preprocess, bwd main, bwd dQ convert, fp8 fwd, fp8 V transpose, d = 256 fwd
+constexpr int kKernelKinds = 7;
+const char* const kKernelNames[kKernelKinds] = {
+    "fa_fwd_kernel",     "fa_bwd_preprocess",  "fa_bwd_main",       "fa_bwd_dq_convert",
+    "fa_fwd_fp8_kernel", "fa_fp8_transpose_v", "fa_fwd_d256_kernel"};
 struct ProfileRec {
   int kind;
   cudaEvent_t start, stop;
@@ -90,6 +91,7 @@ struct DeviceState {
   // threads may launch concurrently; setting an attribute twice is harmless)
   std::atomic<bool> fwd_attr[2][2][2] = {};
   std::atomic<bool> fp8_attr[2] = {};  // [causal]
+  std::atomic<bool> d256_attr[2] = {};  // [causal]
   std::atomic<bool> bwd_attr[2][2][2] = {};
 };
 std::mutex g_mu;
@@ -211,8 +213,8 @@ fa_status check_shape(const Shape& s) {
                    s.B, s.H, s.H_kv, s.N_q, s.N_kv);
   if (s.H % s.H_kv != 0)
     return set_err(FA_ERR_INVALID_ARG, "H=%d is not a multiple of H_kv=%d", s.H, s.H_kv);
-  if (s.d != 64 && s.d != 96 && s.d != 128)
-    return set_err(FA_ERR_UNSUPPORTED, "head dim d=%d not in {64, 96, 128}", s.d);
+  if (s.d != 64 && s.d != 96 && s.d != 128 && s.d != 256)
+    return set_err(FA_ERR_UNSUPPORTED, "head dim d=%d not in {64, 96, 128, 256}", s.d);
   if (s.mask < 0 || s.mask > 2) return set_err(FA_ERR_INVALID_ARG, "mask mode %d unknown", s.mask);
   const long long rows_q = 1LL * s.B * s.H * s.N_q, rows_kv = 1LL * s.B * s.H_kv * s.N_kv;
   if (rows_q >= (1LL << 31) || rows_kv >= (1LL << 31))
@@ -397,9 +399,60 @@ fa_status fwd_dispatch_d(DeviceState* ds, const void* q, const void* k, const vo
                    : launch_fwd<D, CAUSAL, false>(ds, q, k, v, o, lse, s, stream);
 }
 
+// Forward for d = 256 (fa_fwd_d256.cuh): one 128-row query tile per CTA.
+template <bool CAUSAL>
+fa_status launch_fwd_d256(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
+                          float* lse, const Shape& s, cudaStream_t stream) {
+  using L = fa::Fwd256Layout;
+  auto kern = fa::fa_fwd_d256_kernel<CAUSAL>;
+  std::atomic<bool>& attr = ds->d256_attr[CAUSAL];
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncSetAttribute(d256 fwd smem)");
+    cudaFuncAttributes fattr;  // the setmaxnreg split assumes 128 registers per thread
+    e = cudaFuncGetAttributes(&fattr, kern);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncGetAttributes(d256 fwd)");
+    if (fattr.numRegs != 128)
+      return set_err(FA_ERR_CUDA, "d256 forward kernel built with %d registers per thread",
+                     fattr.numRegs);
+    attr = true;
+  }
+  const int BH = s.B * s.H, BHkv = s.B * s.H_kv;
+  CUtensorMap tq, tk, tv, to;
+  fa_status st;
+  if ((st = make_bf16_map(&tq, q, 256, s.N_q, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tk, k, 256, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tv, v, 256, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&to, o, 256, s.N_q, BH, 32)) != FA_OK) return st;
+  fa::FwdParams p;
+  p.lse = lse;
+  p.status = ds->status;
+  p.N = s.N_q;
+  p.N_kv = s.N_kv;
+  p.BH = BH;
+  p.group = s.H / s.H_kv;
+  p.off = s.off();
+  p.n_qblocks = (s.N_q + 127) / 128;
+  p.scale = s.scale;
+  p.scale_log2 = s.scale * 1.4426950408889634f;
+  const long long grid = 1LL * p.n_qblocks * BH;
+  if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  ProfileScope prof(6, stream);
+  kern<<<static_cast<unsigned>(grid), fa::kFwdThreads, L::kAlloc, stream>>>(tq, tk, tv, to, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_fwd (d = 256) launch");
+  return FA_OK;
+}
+
 fa_status fwd_dispatch(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
                        float* lse, const Shape& s, cudaStream_t stream) {
   const bool causal = s.mask != 0;
+  if (s.d == 256) {
+    if (s.dropout) return set_err(FA_ERR_UNSUPPORTED, "dropout is not supported at d = 256");
+    return causal ? launch_fwd_d256<true>(ds, q, k, v, o, lse, s, stream)
+                  : launch_fwd_d256<false>(ds, q, k, v, o, lse, s, stream);
+  }
   if (s.d == 64)
     return causal ? fwd_dispatch_d<64, true>(ds, q, k, v, o, lse, s, stream)
                   : fwd_dispatch_d<64, false>(ds, q, k, v, o, lse, s, stream);
@@ -457,6 +510,8 @@ fa_status bwd_checked(const void* q, const void* k, const void* v, const void* o
                       size_t workspace_bytes, const Shape& s, void* stream) {
   fa_status st = check_shape(s);
   if (st != FA_OK) return st;
+  if (s.d > 128)  // dK and dV of a 128-key tile would need all 512 TMEM columns at d = 256
+    return set_err(FA_ERR_UNSUPPORTED, "the backward supports d <= 128 (got %d)", s.d);
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv)
     return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
   const void* ptrs[10] = {q, k, v, o, dO, lse, dq, dk, dv, workspace};
@@ -565,6 +620,7 @@ fa_status fp8_checked(const void* q8, const void* k8, const void* v8, float qd, 
                       size_t workspace_bytes, void* stream) {
   fa_status st = check_shape(s);
   if (st != FA_OK) return st;
+  if (s.d > 128) return set_err(FA_ERR_UNSUPPORTED, "the FP8 forward supports d <= 128");
   if (!q8 || !k8 || !v8 || !o || !lse) return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
   for (float x : {qd, kd, vd})
     if (!std::isfinite(x) || !(x > 0.f))
@@ -678,7 +734,7 @@ size_t fa_bwd_ex_workspace_size(const fa_attn_shape* shape) {
   if (!shape) return 0;
   const Shape s = from_public(shape);
   const char saved = g_err[0];
-  const bool ok = check_shape(s) == FA_OK;
+  const bool ok = check_shape(s) == FA_OK && s.d <= 128;
   if (saved == '\0') g_err[0] = '\0';
   return ok ? bwd_workspace(s) : 0;
 }
@@ -708,7 +764,7 @@ size_t fa_fwd_fp8_workspace_size(const fa_attn_shape* shape) {
   if (!shape) return 0;
   const Shape s = from_public(shape);
   const char saved = g_err[0];
-  const bool ok = check_shape(s) == FA_OK;
+  const bool ok = check_shape(s) == FA_OK && s.d <= 128;
   if (saved == '\0') g_err[0] = '\0';
   return ok ? fp8_workspace(s) : 0;
 }

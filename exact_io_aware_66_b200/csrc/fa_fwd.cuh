@@ -44,6 +44,8 @@ struct FwdRegs {
   static constexpr uint32_t kMma = kShift ? 80 : 96;
   static_assert(256 * kSoftmax + 128 * kEpilogue + 128 * kMma == kFwdThreads * 128,
                 "forward register split must equal the launch allocation");
+  // the softmax warps raise their count (setmaxnreg.inc), the others lower it (.dec)
+  static_assert(kSoftmax > 128 && kEpilogue < 128 && kMma < 128, "setmaxnreg directions");
 };
 // Running-max update threshold, log2 units (exponentials stay below 2^8 between updates).
 constexpr float kRescaleLog2 = 8.0f;

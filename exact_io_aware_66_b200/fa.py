@@ -82,7 +82,7 @@ def mask_code(causal) -> int:
     raise ValueError(f"unknown mask {causal!r}")
 
 
-KERNEL_KINDS = 6
+KERNEL_KINDS = 7
 
 _lib = None
 

@@ -67,7 +67,9 @@ typedef enum {
  * uses key/value head h / (H / H_kv) (grouped heads; H_kv = 1 is a single shared K/V head),
  * and dk, dv of a key/value head sum over the query heads that share it. A query row that sees
  * no key (FA_MASK_CAUSAL_BOTTOM_RIGHT with N_q > N_kv) gets o = 0, lse = -inf and dq = 0.
- * Limits: d in {64, 96, 128}; all sizes >= 1; B*H*N_q and B*H_kv*N_kv < 2^31. */
+ * Limits: d in {64, 96, 128, 256}; all sizes >= 1; B*H*N_q and B*H_kv*N_kv < 2^31. d = 256 is
+ * supported by the forward only (no dropout): the backward and the FP8 forward return
+ * FA_ERR_UNSUPPORTED for it, and fa_bwd_ex_workspace_size returns 0. */
 typedef struct {
   int B, H, H_kv, N_q, N_kv, d;
   float scale; /* finite, > 0; normally 1/sqrt(d) */
@@ -179,12 +181,12 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_des
  * While enabled on the calling thread, every kernel the library launches is bracketed by a
  * pair of CUDA events recorded on its launch stream. fa_profile_read() waits for those events
  * and writes, per kernel kind k (0 = forward, 1 = backward preprocess, 2 = backward main,
- * 3 = backward dQ conversion, 4 = FP8 forward, 5 = FP8 V transpose; FA_KERNEL_KINDS in
- * total), the number of launches to
+ * 3 = backward dQ conversion, 4 = FP8 forward, 5 = FP8 V transpose, 6 = d = 256 forward;
+ * FA_KERNEL_KINDS in total), the number of launches to
  * launches[k] and their summed device time in milliseconds to ms[k], then forgets them.
  * n is the length of both arrays (>= FA_KERNEL_KINDS). Events are created by the library and
  * reused; no device memory is allocated. */
-#define FA_KERNEL_KINDS 6
+#define FA_KERNEL_KINDS 7
 fa_status fa_profile_enable(int on);
 fa_status fa_profile_read(double* ms, long long* launches, int n);
 /* Name of kernel kind k ("" if out of range). */
