@@ -127,10 +127,27 @@ def default_scale(d: int) -> float:
     return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32).item())
 
 
-def _stream_handle(stream) -> int:
+def _stream_handle(stream, device=None) -> int:
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and isinstance(stream, torch.cuda.Stream) and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _one_device(**tensors) -> torch.device:
+    """The CUDA device that every argument tensor is on. The library launches on the calling
+    thread's current device, so each call below runs with this device made current; tensors on
+    different GPUs are refused here rather than handed to a kernel on the wrong one."""
+    dev = None
+    for name, t in tensors.items():
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other tensors on {dev}")
+    return dev
 
 
 def _dims(x: torch.Tensor):
@@ -157,9 +174,11 @@ def fa_fwd(q, k, v, o, lse, causal: bool = False, scale: float | None = None, st
             raise ValueError(f"{n} shape mismatch")
     if tuple(lse.shape) != (B, H, N):
         raise ValueError("lse must be [B, H, N]")
+    dev = _one_device(q=q, k=k, v=v, o=o, lse=lse)
     ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(lse, "lse", torch.float32)]
     scale = default_scale(d) if scale is None else float(scale)
-    st = lib().fa_fwd(*ptrs, B, H, N, d, scale, int(bool(causal)), _stream_handle(stream))
+    with torch.cuda.device(dev):
+        st = lib().fa_fwd(*ptrs, B, H, N, d, scale, int(bool(causal)), _stream_handle(stream, dev))
     _check("fa_fwd", st)
 
 
@@ -181,10 +200,13 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, causal: bool = False,
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(do, "do"),
             _req(lse, "lse", torch.float32), _req(dq, "dq"), _req(dk, "dk"), _req(dv, "dv")]
+    dev = _one_device(q=q, k=k, v=v, o=o, do=do, lse=lse, dq=dq, dk=dk, dv=dv,
+                      workspace=workspace)
     wbytes = workspace.numel() * workspace.element_size()
     scale = default_scale(d) if scale is None else float(scale)
-    st = lib().fa_bwd(*ptrs, workspace.data_ptr(), wbytes, B, H, N, d, scale, int(bool(causal)),
-                      _stream_handle(stream))
+    with torch.cuda.device(dev):
+        st = lib().fa_bwd(*ptrs, workspace.data_ptr(), wbytes, B, H, N, d, scale,
+                          int(bool(causal)), _stream_handle(stream, dev))
     _check("fa_bwd", st)
 
 
@@ -201,8 +223,11 @@ def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal: bool = False,
         raise ValueError("lse must be [B, H, N]")
     ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(do, "do"),
             _req(lse, "lse", torch.float32), _req(dq, "dq"), _req(dk, "dk"), _req(dv, "dv")]
+    dev = _one_device(q=q, k=k, v=v, o=o, do=do, lse=lse, dq=dq, dk=dk, dv=dv)
     scale = default_scale(d) if scale is None else float(scale)
-    st = lib().fa_bwd_noalloc(*ptrs, B, H, N, d, scale, int(bool(causal)), _stream_handle(stream))
+    with torch.cuda.device(dev):
+        st = lib().fa_bwd_noalloc(*ptrs, B, H, N, d, scale, int(bool(causal)),
+                                  _stream_handle(stream, dev))
     _check("fa_bwd_noalloc", st)
 
 
@@ -251,9 +276,12 @@ def fa_fwd_ex(q, k, v, o, lse, causal=False, scale: float | None = None, stream=
         raise ValueError("o shape mismatch")
     if tuple(lse.shape) != (s.B, s.H, s.N_q):
         raise ValueError("lse must be [B, H, N_q]")
+    dev = _one_device(q=q, k=k, v=v, o=o, lse=lse)
     ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(lse, "lse", torch.float32)]
-    _check("fa_fwd_ex", lib().fa_fwd_ex(*ptrs, ctypes.byref(s), _dropout_arg(dropout),
-                                        _stream_handle(stream)))
+    with torch.cuda.device(dev):
+        st = lib().fa_fwd_ex(*ptrs, ctypes.byref(s), _dropout_arg(dropout),
+                             _stream_handle(stream, dev))
+    _check("fa_fwd_ex", st)
 
 
 def fa_bwd_ex_workspace_size(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int,
@@ -281,9 +309,13 @@ def fa_bwd_ex(q, k, v, o, do, lse, dq, dk, dv, workspace, causal=False,
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ptrs = [_req(q, "q"), _req(k, "k"), _req(v, "v"), _req(o, "o"), _req(do, "do"),
             _req(lse, "lse", torch.float32), _req(dq, "dq"), _req(dk, "dk"), _req(dv, "dv")]
+    dev = _one_device(q=q, k=k, v=v, o=o, do=do, lse=lse, dq=dq, dk=dk, dv=dv,
+                      workspace=workspace)
     wbytes = workspace.numel() * workspace.element_size()
-    _check("fa_bwd_ex", lib().fa_bwd_ex(*ptrs, workspace.data_ptr(), wbytes, ctypes.byref(s),
-                                        _dropout_arg(dropout), _stream_handle(stream)))
+    with torch.cuda.device(dev):
+        st = lib().fa_bwd_ex(*ptrs, workspace.data_ptr(), wbytes, ctypes.byref(s),
+                             _dropout_arg(dropout), _stream_handle(stream, dev))
+    _check("fa_bwd_ex", st)
 
 
 def _req8(x: torch.Tensor, name: str):
@@ -317,12 +349,14 @@ def fa_fwd_fp8(q8, k8, v8, descale, o, lse, causal=False, scale: float | None = 
         workspace = torch.empty(max(16, int(lib().fa_fwd_fp8_workspace_size(ctypes.byref(s)))),
                                 dtype=torch.uint8, device=q8.device)
     qd, kd, vd = (float(x) for x in descale)
+    dev = _one_device(q8=q8, k8=k8, v8=v8, o=o, lse=lse, workspace=workspace)
     ptrs = [_req8(q8, "q8"), _req8(k8, "k8"), _req8(v8, "v8")]
-    _check("fa_fwd_fp8", lib().fa_fwd_fp8(*ptrs, qd, kd, vd, _req(o, "o"),
-                                          _req(lse, "lse", torch.float32), ctypes.byref(s),
-                                          workspace.data_ptr(),
-                                          workspace.numel() * workspace.element_size(),
-                                          _stream_handle(stream)))
+    with torch.cuda.device(dev):
+        st = lib().fa_fwd_fp8(*ptrs, qd, kd, vd, _req(o, "o"), _req(lse, "lse", torch.float32),
+                              ctypes.byref(s), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(),
+                              _stream_handle(stream, dev))
+    _check("fa_fwd_fp8", st)
 
 
 def attention_forward_fp8(q8, k8, v8, descale, causal=False, scale: float | None = None,
