@@ -43,6 +43,7 @@ DEFAULT_WORKLOAD = "causal_train_b4h16n4096d128"
 L2_BYTES = 126 * 1024 * 1024
 FLUSH_BYTES = 512 * 1024 * 1024
 KERNEL_SOURCES = ["exact_io_aware_66_b200/csrc/fa_bwd.cuh", "exact_io_aware_66_b200/csrc/fa_fwd.cuh",
+                  "exact_io_aware_66_b200/csrc/fa_bwd_q128.cuh",
                   "exact_io_aware_66_b200/csrc/fa_fwd_d256.cuh",
                   "exact_io_aware_66_b200/csrc/sm100.cuh", "exact_io_aware_66_b200/csrc/fa_api.cu",
                   "exact_io_aware_66_b200/csrc/dropout.cuh",

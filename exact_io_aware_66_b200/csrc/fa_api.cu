@@ -15,6 +15,7 @@
 
 #include "../../include/fa.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd_q128.cuh"
 #include "fa_fwd_d256.cuh"
 #include "fa_fwd_fp8.cuh"
 #include "fa_fwd.cuh"
@@ -93,6 +94,7 @@ struct DeviceState {
   std::atomic<bool> fp8_attr[2] = {};  // [causal]
   std::atomic<bool> d256_attr[2] = {};  // [causal]
   std::atomic<bool> bwd_attr[2][2][2] = {};
+  std::atomic<bool> bwd128_attr[2] = {};  // [causal]
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -392,6 +394,116 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   return FA_OK;
 }
 
+// Backward at d = 128 (and 96) without dropout: the 128-row query tile kernel
+// (fa_bwd_q128.cuh), between the same preprocess and dQ conversion as launch_bwd.
+template <bool CAUSAL>
+fa_status launch_bwd_q128(DeviceState* ds, const void* q, const void* k, const void* v,
+                          const void* o, const void* dO, const float* lse, void* dq, void* dk,
+                          void* dv, void* workspace, const Shape& s, cudaStream_t stream) {
+  using L = fa::Bwd128Layout;
+  auto kern = fa::fa_bwd_main_q128<CAUSAL>;
+  std::atomic<bool>& attr = ds->bwd128_attr[CAUSAL];
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncSetAttribute(q128 bwd smem)");
+    cudaFuncAttributes fattr;  // the setmaxnreg split assumes 128 registers per thread
+    e = cudaFuncGetAttributes(&fattr, kern);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncGetAttributes(q128 bwd)");
+    if (fattr.numRegs != static_cast<int>(fa::Bwd128Regs::kLaunch))
+      return set_err(FA_ERR_CUDA, "q128 backward kernel built with %d registers per thread",
+                     fattr.numRegs);
+    if (fattr.sharedSizeBytes != 0)
+      return set_err(FA_ERR_CUDA, "q128 backward kernel has %zu bytes of static shared memory",
+                     fattr.sharedSizeBytes);
+    attr = true;
+  }
+  const int BH = s.B * s.H, BHkv = s.B * s.H_kv, N = s.N_q;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(ws);
+  float* Dvec = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_D(BH, N, s.d));
+  float* lse2 = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_lse2(BH, N, s.d));
+  const int n64 = static_cast<int>(fa::bwd_n64(N));
+  const long long rows = 1LL * BH * N;
+
+  CUtensorMap tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv;
+  fa_status st;
+  if ((st = make_bf16_map(&tq, q, s.d, N, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tk, k, s.d, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tv, v, s.d, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdo, dO, s.d, N, BH, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdk, dk, s.d, s.N_kv, BHkv, 32)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdv, dv, s.d, s.N_kv, BHkv, 32)) != FA_OK) return st;
+  // per-row fp32 vectors: [BH][N_q] with a row stride of N64 elements, 128-element boxes
+  if ((st = make_map(&tl, lse2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 128, 1,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
+    return st;
+  if ((st = make_map(&tD, Dvec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 128, 1,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
+    return st;
+  // dQ accumulator: fp32 [BH][N_q][d], reduction boxes of 32 columns x 64 rows
+  if ((st = make_map(&tacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, s.d, N, BH, 32, 64,
+                     CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
+    return st;
+
+  const long long prep_threads = rows * 16;
+  const long long prep_blocks = (prep_threads + fa::kPrepThreads - 1) / fa::kPrepThreads;
+  if (prep_blocks >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  {
+    ProfileScope prof(1, stream);
+    const auto* o16 = static_cast<const __nv_bfloat16*>(o);
+    const auto* do16 = static_cast<const __nv_bfloat16*>(dO);
+    const unsigned nb = static_cast<unsigned>(prep_blocks);
+    if (s.d == 96)
+      fa::fa_bwd_preprocess<96><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc, Dvec,
+                                                                     lse2, rows, N, n64);
+    else
+      fa::fa_bwd_preprocess<128><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc,
+                                                                      Dvec, lse2, rows, N, n64);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_bwd preprocess launch");
+
+  fa::BwdParams p{};
+  p.status = ds->status;
+  p.N = N;
+  p.N_kv = s.N_kv;
+  p.BH_kv = BHkv;
+  p.qgroup = s.H / s.H_kv;
+  p.off = s.off();
+  p.n_kv = (s.N_kv + 127) / 128;
+  p.n_q = (N + 127) / 128;
+  p.d = s.d;
+  {
+    // key/value heads per scheduling group, sized as in launch_bwd
+    const double per_head = static_cast<double>(s.N_kv) * 128 * 4 +
+                            static_cast<double>(p.qgroup) * N * 128 * (2 + 2 + 4);
+    const int g = static_cast<int>(64.0 * 1024 * 1024 / per_head);
+    p.group = g < 1 ? 1 : (g > BHkv ? BHkv : g);
+  }
+  p.scale = s.scale;
+  p.scale_log2 = s.scale * 1.4426950408889634f;
+  const long long grid = 1LL * p.n_kv * BHkv;
+  if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  {
+    ProfileScope prof(2, stream);
+    kern<<<static_cast<unsigned>(grid), fa::kBwdThreads, L::kBytes, stream>>>(
+        tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv, p);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_bwd main (q128) launch");
+
+  const long long n8 = rows * s.d / 8;
+  {
+    ProfileScope prof(3, stream);
+    fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
+        dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_bwd convert launch");
+  return FA_OK;
+}
+
 template <int D, bool CAUSAL>
 fa_status fwd_dispatch_d(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
                          float* lse, const Shape& s, cudaStream_t stream) {
@@ -464,9 +576,12 @@ template <int D, bool CAUSAL>
 fa_status bwd_dispatch_d(DeviceState* ds, const void* q, const void* k, const void* v,
                          const void* o, const void* dO, const float* lse, void* dq, void* dk,
                          void* dv, void* workspace, const Shape& s, cudaStream_t stream) {
-  return s.dropout
-             ? launch_bwd<D, CAUSAL, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream)
-             : launch_bwd<D, CAUSAL, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
+  if (s.dropout)
+    return launch_bwd<D, CAUSAL, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
+  if constexpr (D == 128)
+    return launch_bwd_q128<CAUSAL>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
+  else
+    return launch_bwd<D, CAUSAL, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
 }
 
 fa_status bwd_dispatch(DeviceState* ds, const void* q, const void* k, const void* v, const void* o,
@@ -687,6 +802,7 @@ struct NoAllocDevice {
   void* scratch = nullptr;  // device address of g_noalloc_scratch on this device
   int* status = nullptr;    // device address of g_noalloc_status on this device
   bool bwd_attr[2][2][2] = {};
+  bool bwd128_attr[2] = {};
 };
 
 void copy_flags(std::atomic<bool> (&dst)[2][2][2], const bool (&src)[2][2][2]) {
@@ -873,6 +989,7 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
     local.status = nd.status;
     local.checked = local.is_sm100 = true;
     copy_flags(local.bwd_attr, nd.bwd_attr);
+    for (int c = 0; c < 2; ++c) local.bwd128_attr[c].store(nd.bwd128_attr[c]);
   }
   // The first kernel of the backward rewrites every scratch byte the later ones read (dQ
   // accumulator zeroed, D and -lse*log2e recomputed), so the previous call's contents do not
@@ -882,6 +999,7 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   {
     std::lock_guard<std::mutex> lock(g_mu);
     copy_flags(g_noalloc[dev].bwd_attr, local.bwd_attr);
+    for (int c = 0; c < 2; ++c) g_noalloc[dev].bwd128_attr[c] = local.bwd128_attr[c].load();
   }
   return st;
 }
@@ -913,7 +1031,8 @@ fa_status fa_check_status(void* stream) {
   if (h != 0) {
     e = cudaMemset(ds->status, 0, sizeof(int));
     if (e != cudaSuccess) return cuda_err(e, "clear status word");
-    return set_err(FA_ERR_TIMEOUT, "a bounded in-kernel wait timed out (code %d)", h);
+    return set_err(FA_ERR_TIMEOUT, h == 7 ? "a kernel found its shared memory misaligned (code 7)"
+                                           : "a bounded in-kernel wait timed out (code %d)", h);
   }
   return FA_OK;
 }

@@ -28,8 +28,9 @@
  * Errors. Arguments are validated before anything is launched; a failed check returns a
  * non-zero fa_status, launches nothing, and fa_last_error_string() describes it (thread-local).
  * Every wait inside the kernels is bounded; a wait that times out makes the kernel give up,
- * record FA_ERR_TIMEOUT in the device status word and return. fa_check_status() synchronises
- * the stream, reads and clears that word.
+ * record FA_ERR_TIMEOUT in the device status word and return (a kernel that finds its shared
+ * memory misaligned gives up the same way, with its own code in the message). fa_check_status()
+ * synchronises the stream, reads and clears that word.
  */
 #ifndef FA_H_
 #define FA_H_
