@@ -68,8 +68,10 @@ struct Bwd128Layout {
 };
 static_assert(Bwd128Layout::kBytes <= 227 * 1024, "q128 backward shared memory");
 
-// Register split (setmaxnreg, per warpgroup): two elementwise warpgroups keep a row of 64 fp32
-// probabilities between their two phases; the shares add up to the launch allocation.
+// Register split (setmaxnreg, per warpgroup): the drain warpgroup holds its lanes' 128 dQ^T
+// columns in registers while it stages them; the two elementwise warpgroups (64 fp32
+// probabilities per thread between their two phases) and the MMA/TMA warpgroup give up the
+// difference. The shares add up to the launch allocation.
 struct Bwd128Regs {
   static constexpr uint32_t kLaunch = 128;  // registers per thread at launch (checked on the host)
   static constexpr uint32_t kElem = 120, kDrain = 168, kOther = 104;
