@@ -164,3 +164,14 @@ def test_dropout_validation_without_gpu(lib):
         assert lib.fa_fwd_ex(16, 1 << 16, 2 << 16, 1 << 20, 2 << 20, ctypes.byref(s),
                              ctypes.byref(d), None) == 1
         assert "dropout" in fa.fa_last_error_string()
+
+
+def test_sources_hash_covers_every_library_source():
+    """bench.py's roofline traffic is trusted only while the ncu captures match the sources hash,
+    so the hash must cover every file the library is compiled from."""
+    import bench
+
+    csrc = os.path.join(ROOT, "exact_io_aware_66_b200", "csrc")
+    compiled = {f"exact_io_aware_66_b200/csrc/{fn}" for fn in os.listdir(csrc)
+                if fn.endswith((".cu", ".cuh"))}
+    assert compiled <= set(bench.KERNEL_SOURCES), sorted(compiled - set(bench.KERNEL_SOURCES))
