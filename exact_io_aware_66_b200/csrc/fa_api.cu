@@ -83,6 +83,25 @@ struct ProfileScope {
   }
 };
 
+// ---- failure-detection test hook (fa_debug_stall_next) ----
+// When armed on the calling thread, the next launch of the chosen kernel kind carries a load
+// for its producer to leave out and a short limit for its MMA warp's waits; it is disarmed by
+// that launch.
+struct StallHook {
+  int kind = -1;  // kernel kind (0 forward, 2 backward main) or -1: not armed
+  int skip = 0;
+  unsigned long long limit_ns = 0;
+};
+thread_local StallHook g_stall;
+
+template <class P>
+void apply_stall(int kind, P& p) {
+  if (g_stall.kind != kind) return;
+  p.dbg_skip = g_stall.skip;
+  p.limit_ns = g_stall.limit_ns;
+  g_stall.kind = -1;
+}
+
 constexpr int kMaxDevices = 64;
 struct DeviceState {
   int* status = nullptr;  // device status word
@@ -209,6 +228,16 @@ struct Shape {
   int off() const { return mask == 2 ? N_kv - N_q : 0; }
 };
 
+// Query heads per forward scheduling group: consecutive heads whose K and V (kv_row_bytes per
+// key row of a key/value head, shared by `qgroup` query heads) fill about a quarter of the
+// 126 MB L2, so that K/V tiles are still resident when the group's other query blocks read them.
+int fwd_head_group(const Shape& s, double kv_row_bytes) {
+  const double per_qhead = static_cast<double>(s.N_kv) * kv_row_bytes / (s.H / s.H_kv);
+  const int g = static_cast<int>(32.0 * 1024 * 1024 / per_qhead);
+  const int BH = s.B * s.H;
+  return g < 1 ? 1 : (g > BH ? BH : g);
+}
+
 fa_status check_shape(const Shape& s) {
   if (s.B < 1 || s.H < 1 || s.H_kv < 1 || s.N_q < 1 || s.N_kv < 1)
     return set_err(FA_ERR_INVALID_ARG, "B, H, H_kv, N_q, N_kv must be >= 1 (got %d, %d, %d, %d, %d)",
@@ -281,9 +310,11 @@ fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* 
   p.group = s.H / s.H_kv;
   p.off = s.off();
   p.n_qblocks = (s.N_q + 255) / 256;
+  p.hgroup = fwd_head_group(s, 4.0 * s.d);
   p.scale = s.scale;
   p.scale_log2 = s.scale * 1.4426950408889634f;
   p.drop = s.drop;
+  apply_stall(0, p);
   const long long grid = 1LL * p.n_qblocks * BH;
   if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
   ProfileScope prof(0, stream);
@@ -373,6 +404,7 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   p.scale = s.scale;
   p.scale_log2 = s.scale * 1.4426950408889634f;
   p.drop = s.drop;
+  apply_stall(2, p);
   const long long grid = 1LL * p.n_kv * BHkv;
   if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
   {
@@ -483,6 +515,7 @@ fa_status launch_bwd_q128(DeviceState* ds, const void* q, const void* k, const v
   }
   p.scale = s.scale;
   p.scale_log2 = s.scale * 1.4426950408889634f;
+  apply_stall(2, p);
   const long long grid = 1LL * p.n_kv * BHkv;
   if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
   {
@@ -546,6 +579,7 @@ fa_status launch_fwd_d256(DeviceState* ds, const void* q, const void* k, const v
   p.group = s.H / s.H_kv;
   p.off = s.off();
   p.n_qblocks = (s.N_q + 127) / 128;
+  p.hgroup = fwd_head_group(s, 4.0 * 256);
   p.scale = s.scale;
   p.scale_log2 = s.scale * 1.4426950408889634f;
   const long long grid = 1LL * p.n_qblocks * BH;
@@ -716,6 +750,7 @@ fa_status launch_fwd_fp8(DeviceState* ds, const void* q8, const void* k8, const 
   p.group = s.H / s.H_kv;
   p.off = s.off();
   p.n_qblocks = (s.N_q + 255) / 256;
+  p.hgroup = fwd_head_group(s, 2.0 * s.d);
   p.o_boxes = (s.d + 63) / 64;
   p.scale_log2 = s.scale * 1.4426950408889634f * q_descale * k_descale;
   p.o_scale = v_descale;
@@ -938,6 +973,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   const Shape shape{B, H, H, N, N, d, scale, causal ? 1 : 0};
   fa_status st = check_shape(shape);
   if (st != FA_OK) return st;
+  if (d > 128)  // as bwd_checked: no backward kernel at d = 256 (and no scratch size for it)
+    return set_err(FA_ERR_UNSUPPORTED, "the backward supports d <= 128 (got %d)", d);
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
   if (need > kNoAllocScratchBytes)
     return set_err(FA_ERR_UNSUPPORTED,
@@ -1018,22 +1055,55 @@ fa_status fa_selftest_timeout(int limit_us, void* stream) {
   return FA_OK;
 }
 
+fa_status fa_debug_stall_next(int kind, int skip, int limit_us) {
+  g_err[0] = '\0';
+  if (kind == -1) {
+    g_stall.kind = -1;
+    return FA_OK;
+  }
+  if (kind != 0 && kind != 2)
+    return set_err(FA_ERR_INVALID_ARG, "kind must be 0 (forward), 2 (backward main) or -1");
+  if (skip < 0) return set_err(FA_ERR_INVALID_ARG, "skip must be >= 0 (got %d)", skip);
+  if (limit_us < 1 || limit_us > 10000000)
+    return set_err(FA_ERR_INVALID_ARG, "limit_us must be in [1, 10^7] (got %d)", limit_us);
+  g_stall.kind = kind;
+  g_stall.skip = skip;
+  g_stall.limit_ns = 1000ull * static_cast<unsigned long long>(limit_us);
+  return FA_OK;
+}
+
 fa_status fa_check_status(void* stream) {
   g_err[0] = '\0';
-  fa_status st;
-  DeviceState* ds = device_state(&st);
-  if (!ds) return st;
-  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_err(e, "cudaStreamSynchronize");
-  int h = 0;
-  e = cudaMemcpy(&h, ds->status, sizeof(int), cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess) return cuda_err(e, "read status word");
-  if (h != 0) {
-    e = cudaMemset(ds->status, 0, sizeof(int));
-    if (e != cudaSuccess) return cuda_err(e, "clear status word");
-    return set_err(FA_ERR_TIMEOUT, h == 7 ? "a kernel found its shared memory misaligned (code 7)"
-                                           : "a bounded in-kernel wait timed out (code %d)", h);
+  // Allocates nothing: it reads the words that exist (the allocating entry points' word once
+  // it has been created, and the built-in word of fa_bwd_noalloc once that path is set up),
+  // so callers of fa_bwd_noalloc can use it too.
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_err(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return set_err(FA_ERR_CUDA, "device index %d out of range", dev);
+  int* words[2] = {nullptr, nullptr};
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    words[0] = g_dev[dev].status;
+    if (g_noalloc[dev].ready) words[1] = g_noalloc[dev].status;
   }
+  e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_err(e, "cudaStreamSynchronize");
+  int code = 0;
+  for (int* w : words) {
+    if (!w) continue;
+    int h = 0;
+    e = cudaMemcpy(&h, w, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_err(e, "read status word");
+    if (h != 0) {
+      e = cudaMemset(w, 0, sizeof(int));
+      if (e != cudaSuccess) return cuda_err(e, "clear status word");
+      if (code == 0) code = h;
+    }
+  }
+  if (code != 0)
+    return set_err(FA_ERR_TIMEOUT, code == 7 ? "a kernel found its shared memory misaligned (code 7)"
+                                             : "a bounded in-kernel wait timed out (code %d)", code);
   return FA_OK;
 }
 

@@ -169,6 +169,11 @@ struct BwdParams {
   float scale;
   float scale_log2;
   DropoutParams drop;  // read only by the DROPOUT instantiations
+  // Failure-detection test hook (off by default): the producer never issues the Q tile of
+  // iteration dbg_skip of each CTA, so the MMA warp's wait for it runs out after limit_ns and
+  // the kernel unwinds with FA_ERR_TIMEOUT. limit_ns bounds the MMA warp's waits.
+  int dbg_skip = -1;
+  unsigned long long limit_ns = FA_SPIN_LIMIT_NS;
 };
 
 template <int D, bool CAUSAL, bool DROPOUT>
@@ -495,36 +500,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         umma_commit(bar(L::bQEmpty + st));
         umma_commit(bar(L::bDSFree + b));
       };
-      bool ok = n_i == 0 || mbar_wait(bar(L::bKV), 0, abort_flag);
+      const uint64_t lim = p.limit_ns;
+      bool ok = n_i == 0 || mbar_wait(bar(L::bKV), 0, abort_flag, lim);
       for (int i = 0; i < n_i && ok; ++i) {
         const int b = i & 1, st = i % QS;
-        ok = mbar_wait(bar(L::bQFull + st), (i / QS) & 1, abort_flag) &&
-             (i < 2 || mbar_wait(bar(L::bDQFree + b), ((i >> 1) & 1) ^ 1, abort_flag));
+        ok = mbar_wait(bar(L::bQFull + st), (i / QS) & 1, abort_flag, lim) &&
+             (i < 2 || mbar_wait(bar(L::bDQFree + b), ((i >> 1) & 1) ^ 1, abort_flag, lim));
         if (!ok) break;
         tc_fence_after();
         first_half(i);
         if (i > 0) {
           const int pb = (i - 1) & 1;
-          if (!mbar_wait(bar(L::bEwDone + pb), ((i - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar(L::bEwDone + pb), ((i - 1) >> 1) & 1, abort_flag, lim)) { ok = false; break; }
           tc_fence_after();
           second_half(i - 1);
         }
       }
       if (ok && n_i > 0) {
         const int i = n_i - 1;
-        ok = mbar_wait(bar(L::bEwDone + (i & 1)), (i >> 1) & 1, abort_flag);
+        ok = mbar_wait(bar(L::bEwDone + (i & 1)), (i >> 1) & 1, abort_flag, lim);
         if (ok) {
           tc_fence_after();
           second_half(i);
           umma_commit(bar(L::bAccDone));
         }
       }
-      if (!ok) {
-        fail(p.status, abort_flag, 5);
-        volatile int never = 0;
-        umma_commit(bar(L::bDrain));
-        mbar_wait(bar(L::bDrain), 0, &never);
-      }
+      if (!ok) fail(p.status, abort_flag, 5);
+      // Every MMA this thread issued completes before tensor memory is freed (the drain after a
+      // give-up; on the normal path the epilogue waits for the same products). Bounded wait.
+      volatile int never = 0;
+      umma_commit(bar(L::bDrain));
+      mbar_wait(bar(L::bDrain), 0, &never);
     }
   } else if (warp == 13) {
     // --------------------------------------------------------------------- TMA ----------
@@ -545,6 +551,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           break;
         }
         const int q0 = 64 * q_tile(i), qh = q_head(i);
+        issued = i + 1;
+        if (i == p.dbg_skip) continue;  // (the test hook leaves this tile out)
         mbar_arrive_expect_tx(bar(L::bQFull + st), 2 * L::kQTile + 512);
 #pragma unroll
         for (int bx = 0; bx < L::kBoxes; ++bx) {
@@ -555,14 +563,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         tma_load_3d(sbase + L::kRow + st * 512, &tmLse2, bar(L::bQFull + st), q0, qh, 0);
         tma_load_3d(sbase + L::kRow + st * 512 + 256, &tmD, bar(L::bQFull + st), q0, qh, 0);
-        issued = i + 1;
       }
-      if (*abort_flag) {
-        volatile int never = 0;
-        for (int i = max(0, issued - QS); i < issued; ++i)
-          mbar_wait(bar(L::bQFull + (i % QS)), (i / QS) & 1, &never);
-        if (n_i > 0) mbar_wait(bar(L::bKV), 0, &never);
-      }
+      // Every load issued lands before the CTA can exit, whether or not (or whenever) a role
+      // gives up; the last QS loads are the latest in their stages, so on the normal path these
+      // bounded waits return at once.
+      volatile int never = 0;
+      for (int i = max(0, issued - QS); i < issued; ++i)
+        if (i != p.dbg_skip) mbar_wait(bar(L::bQFull + (i % QS)), (i / QS) & 1, &never);
+      if (n_i > 0) mbar_wait(bar(L::bKV), 0, &never);
     }
   }
   tc_fence_before();

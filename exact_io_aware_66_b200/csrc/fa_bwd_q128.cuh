@@ -404,18 +404,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           umma_ss(tmem + L::tDP, sdesc_advance(dKt_mn, kk * 2048),
                   sdesc_advance(dDS_mn, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
       };
-      bool ok = n_i == 0 || mbar_wait(bar(L::bKV), 0, abort_flag);
+      const uint64_t lim = p.limit_ns;
+      bool ok = n_i == 0 || mbar_wait(bar(L::bKV), 0, abort_flag, lim);
       for (int i = 0; i <= n_i && ok; ++i) {
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
         if (i < n_i) {
-          if (!(ok = mbar_wait(bar(L::bQFull + st), ph, abort_flag))) break;
+          if (!(ok = mbar_wait(bar(L::bQFull + st), ph, abort_flag, lim))) break;
           tc_fence_after();
           mma_s(i);
           umma_commit(bar(L::bSFull));
         }
         if (i > 0) {
-          if (!(ok = mbar_wait(bar(L::bDSDone), (i - 1) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(bar(L::bDSDone), (i - 1) & 1, abort_flag, lim))) break;
           tc_fence_after();
           mma_dk(i - 1);
           umma_commit(bar(L::bQEmpty + ((i - 1) & 1)));
@@ -423,13 +424,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           umma_commit(bar(L::bDQFull));
         }
         if (i < n_i) {
-          if (!(ok = mbar_wait(bar(L::bOFull), i & 1, abort_flag) &&
-                     mbar_wait(bar(L::bPDone), i & 1, abort_flag)))
+          if (!(ok = mbar_wait(bar(L::bOFull), i & 1, abort_flag, lim) &&
+                     mbar_wait(bar(L::bPDone), i & 1, abort_flag, lim)))
             break;
           tc_fence_after();
           mma_dv(i);
           if (i > 0) {
-            if (!(ok = mbar_wait(bar(L::bDQFree), (i - 1) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait(bar(L::bDQFree), (i - 1) & 1, abort_flag, lim))) break;
             tc_fence_after();
           }
           mma_dp();
@@ -438,12 +439,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       if (ok && n_i > 0) umma_commit(bar(L::bAccDone));
-      if (!ok) {
-        fail(p.status, abort_flag, 5);
-        volatile int never = 0;
-        umma_commit(bar(L::bDrain));
-        mbar_wait(bar(L::bDrain), 0, &never);
-      }
+      if (!ok) fail(p.status, abort_flag, 5);
+      // Every MMA this thread issued completes before tensor memory is freed (the drain after a
+      // give-up; on the normal path the epilogue waits for the same products). Bounded wait.
+      volatile int never = 0;
+      umma_commit(bar(L::bDrain));
+      mbar_wait(bar(L::bDrain), 0, &never);
     } else if (warp == 13 && lane == 0) {
       // ------------------------------------------------------------------- TMA ----------
       if (n_i > 0) {
@@ -464,13 +465,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           fail(p.status, abort_flag, 5);
           break;
         }
-        mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTile + 1024);
+        if (i != p.dbg_skip) {  // (the test hook leaves this tile out)
+          mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTile + 1024);
 #pragma unroll
-        for (int bx = 0; bx < 2; ++bx)
-          tma_load_3d(sbase + L::kQ + so + bx * L::kBox, &tmQ, bar(L::bQFull + st), 64 * bx, q0,
-                      qh);
-        tma_load_3d(sbase + L::kRow + st * 1024, &tmLse2, bar(L::bQFull + st), q0, qh, 0);
-        tma_load_3d(sbase + L::kRow + st * 1024 + 512, &tmD, bar(L::bQFull + st), q0, qh, 0);
+          for (int bx = 0; bx < 2; ++bx)
+            tma_load_3d(sbase + L::kQ + so + bx * L::kBox, &tmQ, bar(L::bQFull + st), 64 * bx,
+                        q0, qh);
+          tma_load_3d(sbase + L::kRow + st * 1024, &tmLse2, bar(L::bQFull + st), q0, qh, 0);
+          tma_load_3d(sbase + L::kRow + st * 1024 + 512, &tmD, bar(L::bQFull + st), q0, qh, 0);
+        }
         issued_q = i + 1;
         // dO(i): the single slot frees after dP(i-1)
         if (i > 0 && !mbar_wait(bar(L::bOEmpty), (i - 1) & 1, abort_flag)) {
@@ -483,13 +486,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_3d(sbase + L::kDO + bx * L::kBox, &tmDO, bar(L::bOFull), 64 * bx, q0, qh);
         issued_o = i + 1;
       }
-      if (*abort_flag) {  // let every issued copy land before the CTA exits
-        volatile int never = 0;
-        if (issued_o > 0) mbar_wait(bar(L::bOFull), (issued_o - 1) & 1, &never);
-        for (int i = max(0, issued_q - 2); i < issued_q; ++i)
-          mbar_wait(bar(L::bQFull + (i & 1)), (i >> 1) & 1, &never);
-        if (n_i > 0) mbar_wait(bar(L::bKV), 0, &never);
-      }
+      // Every load issued lands before the CTA can exit, whether or not (or whenever) a role
+      // gives up; these are the latest loads of their slots, so on the normal path the bounded
+      // waits return at once.
+      volatile int never = 0;
+      if (issued_o > 0) mbar_wait(bar(L::bOFull), (issued_o - 1) & 1, &never);
+      for (int i = max(0, issued_q - 2); i < issued_q; ++i)
+        if (i != p.dbg_skip) mbar_wait(bar(L::bQFull + (i & 1)), (i >> 1) & 1, &never);
+      if (n_i > 0) mbar_wait(bar(L::bKV), 0, &never);
     }
   }
   tc_fence_before();

@@ -84,11 +84,32 @@ struct FwdParams {
   int BH;           // batch * query heads
   int group;        // query heads per key/value head (1 unless K/V heads are shared)
   int off;          // causal offset: key j visible to query i iff j <= i + off
-  int n_qblocks;    // ceil(N / 256)
+  int n_qblocks;    // query blocks per head
+  int hgroup;       // query heads per scheduling group (see fwd_work_unit)
   float scale;      // softmax scale
   float scale_log2; // scale * log2(e)
   DropoutParams drop;  // read only by the DROPOUT instantiations
+  // Failure-detection test hook (off by default): the producer never issues K/V load number
+  // dbg_skip of each CTA, so the MMA warp's wait for it runs out after limit_ns and the kernel
+  // unwinds with FA_ERR_TIMEOUT. limit_ns bounds the MMA warp's waits.
+  int dbg_skip = -1;
+  unsigned long long limit_ns = FA_SPIN_LIMIT_NS;
 };
+
+// Work unit of CTA `cta` in a forward grid of n_qblocks * BH CTAs: query block qb of query head
+// bh. Heads are taken in groups of `hgroup` consecutive query heads, sized on the host so that a
+// group's K and V stay in L2 while its CTAs run; inside a group the heaviest query blocks
+// (causal work grows with the block index) come first, cycling over the group's heads
+// (longest-processing-time order).
+__device__ __forceinline__ void fwd_work_unit(int cta, int n_qblocks, int BH, int hgroup, int& qb,
+                                              int& bh) {
+  const int per_group = hgroup * n_qblocks;
+  const int g0 = (cta / per_group) * hgroup;
+  const int r = cta % per_group;
+  const int gcur = min(hgroup, BH - g0);
+  qb = n_qblocks - 1 - r / gcur;
+  bh = g0 + r % gcur;
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -140,10 +161,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Longest-processing-time order: all heads' heaviest query blocks (causal work grows with
-  // the block index) are scheduled first.
-  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x / p.BH);
-  const int bh = static_cast<int>(blockIdx.x % p.BH);
+  int qb, bh;
+  fwd_work_unit(static_cast<int>(blockIdx.x), p.n_qblocks, p.BH, p.hgroup, qb, bh);
   const int bh_kv = bh / p.group;  // key/value head of this query head
   const int q0 = qb * 256;
   const int nkv = (p.N_kv + 127) / 128;
@@ -396,7 +415,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint64_t desc_k0 = sdesc_sw128(sbase + L::kKV, 16, 1024);            // K-major
       const uint64_t desc_v0 = sdesc_sw128(sbase + L::kKV, L::kBoxBytes, 1024);  // MN-major
       auto wait_full = [&](int tt) -> bool {
-        return mbar_wait(bar(L::bKvFull + tt % ST), (tt / ST) & 1, abort_flag);
+        return mbar_wait(bar(L::bKvFull + tt % ST), (tt / ST) & 1, abort_flag, p.limit_ns);
       };
       auto issue_s = [&](int t, int j) {
         const uint64_t a0 = sdesc_advance(desc_q0, t * L::kTileBytes);
@@ -418,7 +437,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           umma_ts(d, a + kk * 8, sdesc_advance(b0, kk * 2048), idesc_pv, 1u);
         umma_commit(bar(L::bODone + t));
       };
-      bool ok = n_t[1] == 0 || (mbar_wait(bar(L::bQ), 0, abort_flag) && wait_full(0));
+      bool ok = n_t[1] == 0 || (mbar_wait(bar(L::bQ), 0, abort_flag, p.limit_ns) && wait_full(0));
       if (ok && n_t[1] > 0) {
         tc_fence_after();
         if (n_t[0] > 0) issue_s(0, 0);
@@ -430,7 +449,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!wait_full(tv)) { ok = false; break; }
         tc_fence_after();
         if (j < n_t[0]) {
-          if (!mbar_wait(bar(L::bPFull + 0), j & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar(L::bPFull + 0), j & 1, abort_flag, p.limit_ns)) { ok = false; break; }
           tc_fence_after();
           issue_pv(0, j);
         }
@@ -440,7 +459,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tc_fence_after();
           if (j + 1 < n_t[0]) issue_s(0, j + 1);
         }
-        if (!mbar_wait(bar(L::bPFull + 1), j & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(L::bPFull + 1), j & 1, abort_flag, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
         issue_pv(1, j);
         umma_commit(bar(L::bKvEmpty + tv % ST));
@@ -449,14 +468,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           umma_commit(bar(L::bKvEmpty + tk % ST));
         }
       }
-      if (!ok) {
-        fail(p.status, abort_flag, 5);
-        // Drain: wait (bounded) until every MMA issued so far has completed before TMEM and
-        // shared memory are released.
-        volatile int never = 0;
-        umma_commit(bar(L::bDrain));
-        mbar_wait(bar(L::bDrain), 0, &never);
-      }
+      if (!ok) fail(p.status, abort_flag, 5);
+      // Every MMA this thread issued completes before tensor memory is freed and the CTA exits
+      // (on the normal path the epilogue waits for the same products; after a give-up this is
+      // the drain). Bounded wait.
+      volatile int never = 0;
+      umma_commit(bar(L::bDrain));
+      mbar_wait(bar(L::bDrain), 0, &never);
     } else if (warp == 13 && lane == 0) {
       // ------------------------------------------------------------------ TMA -------------
       mbar_arrive_expect_tx(bar(L::bQ), 2 * L::kTileBytes);
@@ -477,12 +495,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(L::bKvFull + st), L::kTileBytes);
-          const uint32_t dst = sbase + L::kKV + st * L::kTileBytes;
+          if (tt != p.dbg_skip) {  // (the test hook leaves this load out)
+            mbar_arrive_expect_tx(bar(L::bKvFull + st), L::kTileBytes);
+            const uint32_t dst = sbase + L::kKV + st * L::kTileBytes;
 #pragma unroll
-          for (int b = 0; b < L::kBoxes; ++b)
-            tma_load_3d(dst + b * L::kBoxBytes, w ? &tmV : &tmK, bar(L::bKvFull + st), 64 * b,
-                        128 * j, bh_kv);
+            for (int b = 0; b < L::kBoxes; ++b)
+              tma_load_3d(dst + b * L::kBoxBytes, w ? &tmV : &tmK, bar(L::bKvFull + st), 64 * b,
+                          128 * j, bh_kv);
+          }
           issued = tt + 1;
         }
         if (!ok) {
@@ -490,13 +510,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           break;
         }
       }
-      if (*abort_flag) {
-        // Let the loads already in flight land before shared memory is released.
-        volatile int never = 0;
-        for (int tt = max(0, issued - ST); tt < issued; ++tt)
-          mbar_wait(bar(L::bKvFull + tt % ST), (tt / ST) & 1, &never);
-        mbar_wait(bar(L::bQ), 0, &never);
-      }
+      // Every load issued lands before the CTA can exit, whether or not (or whenever) a role
+      // gives up. The last ST loads are the latest in their stages, so on the normal path these
+      // bounded waits return at once.
+      volatile int never = 0;
+#pragma unroll 1
+      for (int tt = max(0, issued - ST); tt < issued; ++tt)
+        if (tt != p.dbg_skip) mbar_wait(bar(L::bKvFull + tt % ST), (tt / ST) & 1, &never);
+      mbar_wait(bar(L::bQ), 0, &never);
     }
   }
   tc_fence_before();

@@ -85,9 +85,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // longest-processing-time order across heads, as in fa_fwd.cuh
-  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x / p.BH);
-  const int bh = static_cast<int>(blockIdx.x % p.BH);
+  // L2-sized head groups, longest first inside a group, as in fa_fwd.cuh
+  int qb, bh;
+  fwd_work_unit(static_cast<int>(blockIdx.x), p.n_qblocks, p.BH, p.hgroup, qb, bh);
   const int bh_kv = bh / p.group;
   const int q0 = qb * 128;
   const int nkv = (p.N_kv + 127) / 128;

@@ -53,6 +53,7 @@ struct Fp8Params {
   float* lse;
   int* status;
   int N, N_kv, BH, group, off, n_qblocks;
+  int hgroup;        // query heads per scheduling group (fwd_work_unit)
   int o_boxes;       // 64-column boxes of O actually stored: ceil(d / 64)
   float scale_log2;  // softmax scale * log2(e) * q_descale * k_descale
   float o_scale;     // v_descale
@@ -119,8 +120,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x / p.BH);
-  const int bh = static_cast<int>(blockIdx.x % p.BH);
+  int qb, bh;
+  fwd_work_unit(static_cast<int>(blockIdx.x), p.n_qblocks, p.BH, p.hgroup, qb, bh);
   const int bh_kv = bh / p.group;
   const int q0 = qb * 256;
   const int nkv = (p.N_kv + 127) / 128;

@@ -38,6 +38,7 @@ SIGNATURES = {
     "fa_kernel_name": (ctypes.c_char_p, [_I]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_selftest_timeout": (_I, [_I, _P]),
+    "fa_debug_stall_next": (_I, [_I, _I, _I]),
     "fa_fwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "fa_bwd_ex_workspace_size": (_Z, [_P]),
     "fa_bwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P, _P]),
@@ -248,6 +249,13 @@ def fa_selftest_timeout(limit_us: int = 20000, stream=None):
     """Launches the bounded-wait self-test kernel (see include/fa.h); follow with
     fa_check_status(), which must then raise FaError with FA_ERR_TIMEOUT."""
     _check("fa_selftest_timeout", lib().fa_selftest_timeout(int(limit_us), _stream_handle(stream)))
+
+
+def fa_debug_stall_next(kind: int, skip: int = 0, limit_us: int = 20000):
+    """Arms the failure-detection test hook for the next launch of kernel kind `kind` on this
+    thread (0 forward, 2 backward main; -1 disarms): that launch leaves out one load, its wait
+    runs out after limit_us and the call's fa_check_status() raises FA_ERR_TIMEOUT."""
+    _check("fa_debug_stall_next", lib().fa_debug_stall_next(int(kind), int(skip), int(limit_us)))
 
 
 def fa_check_status(stream=None):

@@ -45,15 +45,16 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null or aliasing pointer, non-positive size, bad scale */
-  FA_ERR_UNSUPPORTED = 2, /* head dim not 64/128, sizes beyond the limits below */
+  FA_ERR_UNSUPPORTED = 2, /* head dim or sizes beyond the limits stated below */
   FA_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
   FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (no device, launch error) */
   FA_ERR_TIMEOUT = 5,     /* a bounded in-kernel wait expired (reported by fa_check_status) */
   FA_ERR_WORKSPACE = 6    /* backward workspace missing or smaller than fa_bwd_workspace_size */
 } fa_status;
 
-/* Limits: d in {64, 96, 128} (96 runs the d = 128 kernels on zero-filled columns); B, H, N >= 1;
- * B*H*N < 2^31; B*H*ceil(N/256) < 2^31. */
+/* Limits: d in {64, 96, 128, 256} (96 runs the d = 128 kernels on zero-filled columns; the
+ * backward and the FP8 forward take d <= 128); B, H, N >= 1; B*H*N < 2^31;
+ * B*H*ceil(N/256) < 2^31. */
 
 /* Masks of the extended entry points. */
 typedef enum {
@@ -142,8 +143,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * All calls on a device share the one scratch array, which keeps the last call's contents (each
  * call rewrites what it reads before reading it): calls that overlap on the GPU (different
  * streams, or host threads, without ordering between them) race on it and must be serialised
- * by the caller. A timed-out in-kernel wait (the hang guard) is recorded in a status word
- * built into the library, not in the one fa_check_status reads. */
+ * by the caller. d = 256 is rejected with FA_ERR_UNSUPPORTED, as by fa_bwd. A timed-out
+ * in-kernel wait (the hang guard) is recorded in a status word built into the library, which
+ * fa_check_status reads and clears (it allocates nothing). */
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                          const void* dO, const float* lse, void* dq, void* dk, void* dv, int B,
                          int H, int N, int d, float scale, int causal, void* stream);
@@ -155,8 +157,22 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
  * fa_check_status(stream) returns FA_ERR_TIMEOUT and clears the word. */
 fa_status fa_selftest_timeout(int limit_us, void* stream);
 
-/* Synchronises `stream`, then reads and clears the current device's status word.
- * Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA. */
+/* Failure-detection test hook (off unless called): arms, for the calling thread, the next launch
+ * of kernel kind `kind` (0 = attention forward, 2 = backward main kernel; numbering as in
+ * fa_profile_read). In that launch the TMA producer of every CTA leaves out one load (for the
+ * forward, K/V tile load number `skip` of the CTA; for the backward, the query tile of the
+ * CTA's iteration `skip`), and the MMA warp waits at most limit_us microseconds (1 .. 10^7).
+ * Its wait for the missing tile runs out; the kernel lets the copies and products it issued
+ * finish, frees its tensor memory, records FA_ERR_TIMEOUT in the status word and returns,
+ * without faulting or hanging the GPU. The outputs of that call are undefined; a following
+ * fa_check_status returns FA_ERR_TIMEOUT. The launch disarms the hook; kind = -1 disarms it
+ * without a launch. A CTA that issues fewer loads than `skip` runs normally. */
+fa_status fa_debug_stall_next(int kind, int skip, int limit_us);
+
+/* Synchronises `stream`, then reads and clears the current device's status words: the one
+ * the allocating entry points write (if it has been created) and the one built into the
+ * library for fa_bwd_noalloc (if that entry point has been set up on this device). Allocates
+ * no device memory. Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA. */
 fa_status fa_check_status(void* stream);
 
 /* FP8 forward: q8, k8, v8 hold E4M3 codes (OCP 8-bit floating point, the "e4m3fn" encoding:

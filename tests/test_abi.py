@@ -175,3 +175,23 @@ def test_sources_hash_covers_every_library_source():
     compiled = {f"exact_io_aware_66_b200/csrc/{fn}" for fn in os.listdir(csrc)
                 if fn.endswith((".cu", ".cuh"))}
     assert compiled <= set(bench.KERNEL_SOURCES), sorted(compiled - set(bench.KERNEL_SOURCES))
+
+
+def test_debug_stall_hook_validation_without_gpu(lib):
+    assert lib.fa_debug_stall_next(1, 0, 1000) == 1  # only the forward (0) and backward main (2)
+    assert lib.fa_debug_stall_next(0, -1, 1000) == 1
+    assert lib.fa_debug_stall_next(2, 0, 0) == 1
+    assert lib.fa_debug_stall_next(2, 0, 10 ** 8) == 1
+    assert lib.fa_debug_stall_next(0, 3, 20000) == 0
+    assert lib.fa_debug_stall_next(-1, 0, 0) == 0  # disarm
+
+
+def test_noalloc_rejects_d256_without_gpu(lib):
+    """No backward kernel exists at d = 256: fa_bwd_noalloc refuses it before any CUDA call, so
+    its scratch-size check never sees a size it was not written for."""
+    fake = 1 << 24
+    for B, H, N in ((1, 1, 128), (4, 16, 4096)):
+        st = lib.fa_bwd_noalloc(fake, fake * 2, fake * 3, fake * 4, fake * 5, fake * 6, fake * 7,
+                                fake * 8, fake * 9, B, H, N, 256, 0.0625, 1, None)
+        assert st == 2
+        assert "d <= 128" in fa.fa_last_error_string()

@@ -11,7 +11,7 @@ import oracle
 from exact_io_aware_66_b200 import fa
 from exact_io_aware_66_b200.workloads import (WORKLOADS, make_inputs, sampled_keys, sampled_rows,
                                               workload_inputs)
-from parity import TOL_GRAD_REL, assert_grad_ok, grad_rel_error, to64
+from parity import TOL_GRAD_REL, assert_fwd_ok, assert_grad_ok, fwd_errors, grad_rel_error, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -41,31 +41,26 @@ def test_bwd_small_full_compare(shape, causal):
         assert_grad_ok(g, r, f"{shape} causal={causal} {n}")
 
 
-def _head_subset(w, n_heads, seed):
-    rng = np.random.Generator(np.random.PCG64(w.seed + seed))
-    return [divmod(int(t), w.H) for t in rng.choice(w.B * w.H, size=n_heads, replace=False)]
-
-
 @pytest.mark.parametrize("name", ["train_b8h16n2048d64", "causal_train_b4h16n4096d128"])
-def test_bwd_full_size_whole_heads(name):
-    """Full-size training workloads in the bench's launch configuration: dQ, dK, dV of whole
-    seeded heads against the oracle, and dQ of sampled rows across every head."""
+def test_fwd_bwd_full_size_every_element(name):
+    """The two full-size training workloads (B8 H16 N2048 d64 non-causal; B4 H16 N4096 d128
+    causal), in the bench's launch configuration: every element of O, lse, dQ, dK and dV of
+    every head against the oracle. O must meet max-abs 1e-2 and mean-abs 1e-3 on every element
+    (no element may fall back to the bf16-format check), lse 1e-3, gradients 2e-2 relative."""
     w = WORKLOADS[name]
     x = workload_inputs(w)
-    _, _, dq, dk, dv = _fwd_bwd(x, w.causal)
-    for g in (dq, dk, dv):
-        assert torch.isfinite(g).all()
-    dq64, dk64, dv64 = to64(dq), to64(dk), to64(dv)
-    for b, h in _head_subset(w, 2, 3000):
-        ref = oracle.attention_backward(to64(x["q"][b, h]), to64(x["k"][b, h]), to64(x["v"][b, h]),
-                                        to64(x["do"][b, h]), w.scale, w.causal)
-        for g, r, n in zip((dq64[b, h], dk64[b, h], dv64[b, h]), ref, ("dQ", "dK", "dV")):
-            assert_grad_ok(g, r, f"{name} head ({b},{h}) {n}")
-    rows = sampled_rows(w, 256)
-    q, k, v, do = (x[n].float().numpy() for n in ("q", "k", "v", "do"))
-    _, _, dq_ref = oracle.attention_rows(q, k, v, w.scale, w.causal, rows, do=do)
-    idx = tuple(np.array(rows).T)
-    assert grad_rel_error(dq64[idx], dq_ref) <= TOL_GRAD_REL
+    o, lse, dq, dk, dv = _fwd_bwd(x, w.causal)
+    dq_r, dk_r, dv_r, o_r, lse_r = oracle.attention_backward(
+        to64(x["q"]), to64(x["k"]), to64(x["v"]), to64(x["do"]), w.scale, w.causal,
+        return_forward=True)
+    err = fwd_errors(o, lse, o_r, lse_r)
+    assert err["format_limited"] == 0, f"{name}: {err['format_limited']} elements with |O| >= 4"
+    assert err["o_max"] <= 1e-2
+    assert_fwd_ok(err, name)
+    for g, r, n in zip((dq, dk, dv), (dq_r, dk_r, dv_r), ("dQ", "dK", "dV")):
+        rel = assert_grad_ok(g, r, f"{name} {n}")
+        print(f"[parity] {name} {n}: relative max-norm error {rel:.3e}, "
+              f"mean-abs {float(np.abs(to64(g) - r).mean()):.3e}")
 
 
 def test_bwd_long_sequence_sampled():

@@ -36,6 +36,8 @@ CASES = [  # (B, H, H_kv, N_q, N_kv, d, mask)
     (1, 2, 2, 300, 300, 96, False),             # d = 96: the d = 128 kernels, zero-filled
     (2, 4, 2, 513, 513, 96, True),
     (1, 2, 1, 100, 700, 96, "bottom_right"),
+    (1, 2, 2, 200, 600, 128, True),             # d = 128: key tiles 2..4 seen by no query
+    (1, 2, 1, 130, 520, 96, True),              # d = 96, grouped: keys 130.. seen by no query
 ]
 
 

@@ -46,14 +46,15 @@ def test_fwd_first_config_full():
     o_ref, lse_ref = oracle.attention_forward(to64(x["q"]), to64(x["k"]), to64(x["v"]), w.scale,
                                               w.causal)
     err = fwd_errors(o, lse, o_ref, lse_ref)
+    assert err["format_limited"] == 0
     assert_fwd_ok(err, w.name)
 
 
-@pytest.mark.parametrize("name", ["train_b8h16n2048d64", "causal_train_b4h16n4096d128",
-                                  "causal_train_b1h16n16384d128", "causal_fwd_b1h8n131072d128"])
+@pytest.mark.parametrize("name", ["causal_train_b1h16n16384d128", "causal_fwd_b1h8n131072d128"])
 def test_fwd_full_size_sampled_rows(name):
-    """Full-size workloads, same launch configuration as the bench: sampled query rows
-    (512, or 256 at N = 131072) against the oracle, and every output finite."""
+    """The two long-sequence workloads, same launch configuration as the bench: sampled query
+    rows (512, or 256 at N = 131072) against the oracle, and every output finite. (The N = 2048
+    and N = 4096 workloads are compared element by element in test_bwd_gpu.py.)"""
     w = WORKLOADS[name]
     x = workload_inputs(w, with_do=False)
     o, lse = _run(x, w.causal)
@@ -66,6 +67,7 @@ def test_fwd_full_size_sampled_rows(name):
     o_s = to64(o)[idx]
     l_s = to64(lse)[idx]
     err = fwd_errors(o_s, l_s, o_ref, lse_ref)
+    assert err["format_limited"] == 0, f"{name}: {err['format_limited']} elements with |O| >= 4"
     assert_fwd_ok(err, name)
 
 

@@ -54,3 +54,14 @@ def test_noalloc_rejects_sizes_beyond_builtin_scratch():
                                  fake * 7, fake * 8, fake * 9, B, H, N, d, 0.088, 1, None)
     assert st == 2
     assert "built into the library" in fa.fa_last_error_string()
+
+
+def test_noalloc_rejects_d256_before_any_launch():
+    """d = 256 has no backward kernel: the call is refused with FA_ERR_UNSUPPORTED before the
+    scratch-size check and before any launch (the pointers are never touched)."""
+    fake = 1 << 24
+    for B, H, N in ((1, 1, 128), (4, 16, 4096)):
+        st = fa.lib().fa_bwd_noalloc(fake, fake * 2, fake * 3, fake * 4, fake * 5, fake * 6,
+                                     fake * 7, fake * 8, fake * 9, B, H, N, 256, 0.0625, 1, None)
+        assert st == 2
+        assert "d <= 128" in fa.fa_last_error_string()
