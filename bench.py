@@ -17,7 +17,10 @@ FLOPs counted as for bf16, the roofline against twice the measured bf16 peak —
 FP8/bf16 ratio). ``--dropout P`` runs the same step with dropout probability P on the attention probabilities
 (fa_fwd_ex / fa_bwd_ex, a new Philox offset every step); the FLOP count is unchanged.
 ``--impl reference`` times the fp64 CPU oracle on the host instead, on bounded samples of the
-same workload.
+same workload. A single-GPU run of the default workload also times, after the headline, the
+metric's other N >= 4096 configurations (B1 H16 N16384 d128 causal forward + backward, B1 H8
+N131072 d128 causal forward; 5 steps each after 3 warm-up, L2 flushed) and reports them under
+``per_config`` (``--no-per-config`` skips this).
 """
 
 from __future__ import annotations
@@ -69,6 +72,12 @@ def load_peaks() -> dict:
     except Exception:
         return {"bf16_burst": 1590.0, "bf16_sustained": 1400.0, "hbm_gbs": 6650.0,
                 "source": "fallback"}
+
+
+def peak_label(peaks: dict, kind: str) -> str:
+    if peaks["source"] == "measured":
+        return f"measured bf16 {kind} (MEASURED_PEAKS.json)"
+    return f"fallback bf16 {kind} (no MEASURED_PEAKS.json)"
 
 
 def _code_only(src: str) -> str:
@@ -321,6 +330,63 @@ def workload_config(w, world, dropout: float = 0.0, fp8: bool = False) -> dict:
 
 
 # --------------------------------------------------------------------------------------------
+# The other target configurations of the metric's N range, timed beside the headline
+# --------------------------------------------------------------------------------------------
+PER_CONFIG = ("causal_train_b1h16n16384d128", "causal_fwd_b1h8n131072d128")
+
+
+def time_config(name: str, dev, steps: int, warmup: int, peaks: dict) -> dict:
+    """Forward (and backward, if the workload has one) of workload `name` through the C ABI,
+    inputs resident, L2 flushed before every step; per-pass device time from the library's own
+    per-kernel events. Returns TFLOP/s and fractions of the measured burst peak."""
+    from exact_io_aware_66_b200 import fa
+
+    w = WORKLOADS[name]
+    x = workload_inputs(w)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    if w.backward:
+        do = x["do"].to(dev)
+        ws = torch.empty(fa.fa_bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8,
+                         device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    del x
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        fa.fa_fwd(q, k, v, o, lse, w.causal, None, stream)
+        if w.backward:
+            fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, w.causal, None, stream)
+
+    for _ in range(warmup):
+        step()
+    fa.fa_check_status(stream)
+    fa.fa_profile_read()
+    fa.fa_profile_enable(True)
+    for _ in range(steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    fa.fa_profile_enable(False)
+    prof = fa.fa_profile_read()
+    fa.fa_check_status(stream)
+    fwd_ms = prof["fa_fwd_kernel"][1] / steps
+    out = {"B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "steps": steps,
+           "fwd_tflops": w.fwd_flops() / (fwd_ms / 1e3) / 1e12}
+    out["fwd_frac_of_peak"] = out["fwd_tflops"] / peaks["bf16_burst"]
+    if w.backward:
+        bwd_ms = sum(prof[n][1] for n in ("fa_bwd_preprocess", "fa_bwd_main",
+                                           "fa_bwd_dq_convert")) / steps
+        out["bwd_tflops"] = w.bwd_flops() / (bwd_ms / 1e3) / 1e12
+        out["fwd_bwd_tflops"] = (w.fwd_flops() + w.bwd_flops()) / ((fwd_ms + bwd_ms) / 1e3) / 1e12
+        out["fwd_bwd_frac_of_peak"] = out["fwd_bwd_tflops"] / peaks["bf16_burst"]
+    out["peak_source"] = peak_label(peaks, "burst")
+    return out
+
+
+# --------------------------------------------------------------------------------------------
 # Our arm
 # --------------------------------------------------------------------------------------------
 def main():
@@ -334,6 +400,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dropout", type=float, default=0.0)
     ap.add_argument("--fp8", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip timing the other N >= 4096 configurations beside the headline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -441,8 +509,7 @@ def main():
     avg_ms = kern[dom]["ms"] / kern[dom]["launches"]
     sustained = ms_total > 1000
     peak = peaks["bf16_sustained"] if sustained else peaks["bf16_burst"]
-    peak_source = (f"{peaks['source']} bf16 {'sustained' if sustained else 'burst'} "
-                   f"(MEASURED_PEAKS.json)")
+    peak_source = peak_label(peaks, "sustained" if sustained else "burst")
     if dom == "fa_fwd_fp8_kernel":  # E4M3 contraction: nominal FP8/bf16 dense ratio 4.5/2.25
         peak *= 2.0
         peak_source += " x 2 (nominal fp8/bf16 dense ratio)"
@@ -522,6 +589,15 @@ def main():
            "steps": args.e2e_steps,
            "pipeline": "h2d / kernels / d2h on three streams, two device buffer sets"}
 
+    # the metric's other target configurations (N = 16384 fwd+bwd, N = 131072 fwd), timed on
+    # rank 0 of a single-GPU run of the default workload
+    per_config = None
+    if (rank == 0 and world == 1 and not args.no_per_config and args.workload == DEFAULT_WORKLOAD
+            and not args.fp8 and args.dropout == 0):
+        del host_in, dev_in, dev_out, host_out
+        per_config = {name: time_config(name, dev, 5, 3, peaks) for name in PER_CONFIG}
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, x, dropout=args.dropout, fp8=args.fp8)
@@ -541,10 +617,11 @@ def main():
             "frac_of_peak": {"fwd+bwd": value / world / peaks["bf16_burst"],
                              "fwd": (w.fwd_flops() / (fwd_ms / 1e3) / 1e12) / peaks["bf16_burst"]
                              if fwd_ms else None,
-                             "peak": peaks["bf16_burst"], "peak_source":
-                                 f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"},
+                             "peak": peaks["bf16_burst"],
+                             "peak_source": peak_label(peaks, "burst")},
             "roofline": roofline,
             "kernels": kern,
+            "per_config": per_config,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
