@@ -48,6 +48,7 @@ FLUSH_BYTES = 512 * 1024 * 1024
 KERNEL_SOURCES = ["exact_io_aware_66_b200/csrc/fa_bwd.cuh", "exact_io_aware_66_b200/csrc/fa_fwd.cuh",
                   "exact_io_aware_66_b200/csrc/fa_bwd_q128.cuh",
                   "exact_io_aware_66_b200/csrc/fa_fwd_d256.cuh",
+                  "exact_io_aware_66_b200/csrc/fa_bwd_d256.cuh",
                   "exact_io_aware_66_b200/csrc/sm100.cuh", "exact_io_aware_66_b200/csrc/fa_api.cu",
                   "exact_io_aware_66_b200/csrc/dropout.cuh",
                   "exact_io_aware_66_b200/csrc/fa_fwd_fp8.cuh"]
@@ -501,11 +502,17 @@ def main():
                  for n in ("fa_fwd_kernel", "fa_fwd_d256_kernel", "fa_fwd_fp8_kernel",
                            "fa_fp8_transpose_v")) / args.steps
     bwd_ms = sum(kern.get(n, {}).get("ms", 0.0)
-                 for n in ("fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert")) / args.steps
+                 for n in ("fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert",
+                           "fa_bwd_d256_dv", "fa_bwd_d256_dkdq")) / args.steps
     peaks = load_peaks()
     dom = max(kern, key=lambda n: kern[n]["ms"])
+    # algorithmic FLOPs per launch of each main kernel; the d = 256 backward splits its five
+    # products over two passes (the dV pass: dV; the dK/dQ pass: dP, dK, dQ; S in both), so each
+    # is credited with its share of the backward's 2.5 x forward
     dom_flops = {"fa_fwd_kernel": w.fwd_flops(), "fa_bwd_main": w.bwd_flops(),
-                 "fa_fwd_fp8_kernel": w.fwd_flops(), "fa_fwd_d256_kernel": w.fwd_flops()}.get(dom)
+                 "fa_fwd_fp8_kernel": w.fwd_flops(), "fa_fwd_d256_kernel": w.fwd_flops(),
+                 "fa_bwd_d256_dv": w.bwd_flops() * 1.0 / 5.0,
+                 "fa_bwd_d256_dkdq": w.bwd_flops() * 4.0 / 5.0}.get(dom)
     avg_ms = kern[dom]["ms"] / kern[dom]["launches"]
     sustained = ms_total > 1000
     peak = peaks["bf16_sustained"] if sustained else peaks["bf16_burst"]

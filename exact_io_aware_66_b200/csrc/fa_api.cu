@@ -15,6 +15,7 @@
 
 #include "../../include/fa.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd_d256.cuh"
 #include "fa_bwd_q128.cuh"
 #include "fa_fwd_d256.cuh"
 #include "fa_fwd_fp8.cuh"
@@ -37,11 +38,13 @@ fa_status cuda_err(cudaError_t e, const char* what) {
 }
 
 // ---- optional per-kernel device timing (fa_profile_enable / fa_profile_read) ----
-// fwd, bwd preprocess, bwd main, bwd dQ convert, fp8 fwd, fp8 V transpose, d = 256 fwd
-constexpr int kKernelKinds = 7;
+// fwd, bwd preprocess, bwd main, bwd dQ convert, fp8 fwd, fp8 V transpose, d = 256 fwd,
+// d = 256 bwd dV pass, d = 256 bwd dK/dQ pass
+constexpr int kKernelKinds = 9;
 const char* const kKernelNames[kKernelKinds] = {
     "fa_fwd_kernel",     "fa_bwd_preprocess",  "fa_bwd_main",       "fa_bwd_dq_convert",
-    "fa_fwd_fp8_kernel", "fa_fp8_transpose_v", "fa_fwd_d256_kernel"};
+    "fa_fwd_fp8_kernel", "fa_fp8_transpose_v", "fa_fwd_d256_kernel", "fa_bwd_d256_dv",
+    "fa_bwd_d256_dkdq"};
 struct ProfileRec {
   int kind;
   cudaEvent_t start, stop;
@@ -114,6 +117,7 @@ struct DeviceState {
   std::atomic<bool> d256_attr[2] = {};  // [causal]
   std::atomic<bool> bwd_attr[2][2][2] = {};
   std::atomic<bool> bwd128_attr[2] = {};  // [causal]
+  std::atomic<bool> bwd256_attr[2] = {};  // [causal]
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -537,6 +541,114 @@ fa_status launch_bwd_q128(DeviceState* ds, const void* q, const void* k, const v
   return FA_OK;
 }
 
+// Backward at d = 256 (fa_bwd_d256.cuh): preprocess, the dV pass, the dK/dQ pass, dQ conversion.
+template <bool CAUSAL>
+fa_status launch_bwd_d256(DeviceState* ds, const void* q, const void* k, const void* v,
+                          const void* o, const void* dO, const float* lse, void* dq, void* dk,
+                          void* dv, void* workspace, const Shape& s, cudaStream_t stream) {
+  using LA = fa::Bwd256DvLayout;
+  using LB = fa::Bwd256DkdqLayout;
+  auto kern_a = fa::fa_bwd_d256_dv<CAUSAL>;
+  auto kern_b = fa::fa_bwd_d256_dkdq<CAUSAL>;
+  std::atomic<bool>& attr = ds->bwd256_attr[CAUSAL];
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern_a, cudaFuncAttributeMaxDynamicSharedMemorySize, LA::kAlloc);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncSetAttribute(d256 bwd dV smem)");
+    e = cudaFuncSetAttribute(kern_b, cudaFuncAttributeMaxDynamicSharedMemorySize, LB::kAlloc);
+    if (e != cudaSuccess) return cuda_err(e, "cudaFuncSetAttribute(d256 bwd dK/dQ smem)");
+    attr = true;
+  }
+  const int BH = s.B * s.H, BHkv = s.B * s.H_kv, N = s.N_q;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(ws);
+  float* Dvec = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_D(BH, N, 256));
+  float* lse2 = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_lse2(BH, N, 256));
+  const int n64 = static_cast<int>(fa::bwd_n64(N));
+  const long long rows = 1LL * BH * N;
+
+  CUtensorMap tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv;
+  fa_status st;
+  if ((st = make_bf16_map(&tq, q, 256, N, BH, 64)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tk, k, 256, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tv, v, 256, s.N_kv, BHkv, 128)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdo, dO, 256, N, BH, 64)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdk, dk, 256, s.N_kv, BHkv, 32)) != FA_OK) return st;
+  if ((st = make_bf16_map(&tdv, dv, 256, s.N_kv, BHkv, 32)) != FA_OK) return st;
+  // per-row fp32 vectors: [BH][N_q] with a row stride of N64 elements, 64-element boxes
+  if ((st = make_map(&tl, lse2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 64, 1,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
+    return st;
+  if ((st = make_map(&tD, Dvec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 64, 1,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
+    return st;
+  // dQ accumulator: fp32 [BH][N_q][256], reduction boxes of 32 columns x 32 rows
+  if ((st = make_map(&tacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 256, N, BH, 32, 32,
+                     CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
+    return st;
+
+  const long long prep_threads = rows * 32;
+  const long long prep_blocks = (prep_threads + fa::kPrepThreads - 1) / fa::kPrepThreads;
+  if (prep_blocks >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  {
+    ProfileScope prof(1, stream);
+    fa::fa_bwd_preprocess<256><<<static_cast<unsigned>(prep_blocks), fa::kPrepThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dq_acc,
+        Dvec, lse2, rows, N, n64);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_bwd preprocess launch");
+
+  fa::BwdParams p{};
+  p.status = ds->status;
+  p.N = N;
+  p.N_kv = s.N_kv;
+  p.BH_kv = BHkv;
+  p.qgroup = s.H / s.H_kv;
+  p.off = s.off();
+  p.n_kv = (s.N_kv + 127) / 128;
+  p.n_q = (N + 63) / 64;
+  p.d = 256;
+  {
+    // key/value heads per scheduling group, sized as in launch_bwd
+    const double per_head = static_cast<double>(s.N_kv) * 256 * 4 +
+                            static_cast<double>(p.qgroup) * N * 256 * (2 + 2 + 4);
+    const int g = static_cast<int>(64.0 * 1024 * 1024 / per_head);
+    p.group = g < 1 ? 1 : (g > BHkv ? BHkv : g);
+  }
+  p.scale = s.scale;
+  p.scale_log2 = s.scale * 1.4426950408889634f;
+  apply_stall(2, p);
+  const long long grid = 1LL * p.n_kv * BHkv;
+  if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  {
+    ProfileScope prof(7, stream);
+    kern_a<<<static_cast<unsigned>(grid), fa::kBwdThreads, LA::kAlloc, stream>>>(tq, tk, tdo, tl,
+                                                                                 tdv, p);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_bwd (d = 256) dV pass launch");
+  p.dbg_skip = -1;  // the test hook applies to the first pass only
+  p.limit_ns = FA_SPIN_LIMIT_NS;
+  {
+    ProfileScope prof(8, stream);
+    kern_b<<<static_cast<unsigned>(grid), fa::kBwdThreads, LB::kAlloc, stream>>>(
+        tq, tk, tv, tdo, tl, tD, tacc, tdk, p);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_bwd (d = 256) dK/dQ pass launch");
+
+  const long long n8 = rows * 256 / 8;
+  {
+    ProfileScope prof(3, stream);
+    fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
+        dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_err(e, "fa_bwd convert launch");
+  return FA_OK;
+}
+
 template <int D, bool CAUSAL>
 fa_status fwd_dispatch_d(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
                          float* lse, const Shape& s, cudaStream_t stream) {
@@ -622,6 +734,11 @@ fa_status bwd_dispatch(DeviceState* ds, const void* q, const void* k, const void
                        const void* dO, const float* lse, void* dq, void* dk, void* dv,
                        void* workspace, const Shape& s, cudaStream_t stream) {
   const bool causal = s.mask != 0;
+  if (s.d == 256) {
+    if (s.dropout) return set_err(FA_ERR_UNSUPPORTED, "dropout is not supported at d = 256");
+    return causal ? launch_bwd_d256<true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream)
+                  : launch_bwd_d256<false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
+  }
   if (s.d == 64)
     return causal ? bwd_dispatch_d<64, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream)
                   : bwd_dispatch_d<64, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
@@ -659,8 +776,6 @@ fa_status bwd_checked(const void* q, const void* k, const void* v, const void* o
                       size_t workspace_bytes, const Shape& s, void* stream) {
   fa_status st = check_shape(s);
   if (st != FA_OK) return st;
-  if (s.d > 128)  // dK and dV of a 128-key tile would need all 512 TMEM columns at d = 256
-    return set_err(FA_ERR_UNSUPPORTED, "the backward supports d <= 128 (got %d)", s.d);
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv)
     return set_err(FA_ERR_INVALID_ARG, "null pointer argument");
   const void* ptrs[10] = {q, k, v, o, dO, lse, dq, dk, dv, workspace};
@@ -838,6 +953,7 @@ struct NoAllocDevice {
   int* status = nullptr;    // device address of g_noalloc_status on this device
   bool bwd_attr[2][2][2] = {};
   bool bwd128_attr[2] = {};
+  bool bwd256_attr[2] = {};
 };
 
 void copy_flags(std::atomic<bool> (&dst)[2][2][2], const bool (&src)[2][2][2]) {
@@ -877,7 +993,7 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 96 && d != 128)) return 0;
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 96 && d != 128 && d != 256)) return 0;
   return fa::bwd_workspace_bytes(static_cast<size_t>(B) * H, N, d);
 }
 
@@ -885,7 +1001,7 @@ size_t fa_bwd_ex_workspace_size(const fa_attn_shape* shape) {
   if (!shape) return 0;
   const Shape s = from_public(shape);
   const char saved = g_err[0];
-  const bool ok = check_shape(s) == FA_OK && s.d <= 128;
+  const bool ok = check_shape(s) == FA_OK;
   if (saved == '\0') g_err[0] = '\0';
   return ok ? bwd_workspace(s) : 0;
 }
@@ -973,8 +1089,6 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   const Shape shape{B, H, H, N, N, d, scale, causal ? 1 : 0};
   fa_status st = check_shape(shape);
   if (st != FA_OK) return st;
-  if (d > 128)  // as bwd_checked: no backward kernel at d = 256 (and no scratch size for it)
-    return set_err(FA_ERR_UNSUPPORTED, "the backward supports d <= 128 (got %d)", d);
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
   if (need > kNoAllocScratchBytes)
     return set_err(FA_ERR_UNSUPPORTED,
@@ -1026,7 +1140,10 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
     local.status = nd.status;
     local.checked = local.is_sm100 = true;
     copy_flags(local.bwd_attr, nd.bwd_attr);
-    for (int c = 0; c < 2; ++c) local.bwd128_attr[c].store(nd.bwd128_attr[c]);
+    for (int c = 0; c < 2; ++c) {
+      local.bwd128_attr[c].store(nd.bwd128_attr[c]);
+      local.bwd256_attr[c].store(nd.bwd256_attr[c]);
+    }
   }
   // The first kernel of the backward rewrites every scratch byte the later ones read (dQ
   // accumulator zeroed, D and -lse*log2e recomputed), so the previous call's contents do not
@@ -1036,7 +1153,10 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   {
     std::lock_guard<std::mutex> lock(g_mu);
     copy_flags(g_noalloc[dev].bwd_attr, local.bwd_attr);
-    for (int c = 0; c < 2; ++c) g_noalloc[dev].bwd128_attr[c] = local.bwd128_attr[c].load();
+    for (int c = 0; c < 2; ++c) {
+      g_noalloc[dev].bwd128_attr[c] = local.bwd128_attr[c].load();
+      g_noalloc[dev].bwd256_attr[c] = local.bwd256_attr[c].load();
+    }
   }
   return st;
 }

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kPrepThreads)
                       const float* __restrict__ lse, float* __restrict__ dq_acc,
                       float* __restrict__ Dvec, float* __restrict__ lse2, long long rows, int N,
                       int n64) {
-  constexpr int TPR = D <= 64 ? 8 : 16;  // threads per row
+  constexpr int TPR = D <= 64 ? 8 : (D <= 128 ? 16 : 32);  // threads per row
   static_assert(D % 8 == 0 && D / 8 <= TPR, "preprocess row split");
   const long long t = static_cast<long long>(blockIdx.x) * kPrepThreads + threadIdx.x;
   const long long row = t / TPR;

@@ -83,7 +83,7 @@ def mask_code(causal) -> int:
     raise ValueError(f"unknown mask {causal!r}")
 
 
-KERNEL_KINDS = 7
+KERNEL_KINDS = 9
 
 _lib = None
 

@@ -52,9 +52,10 @@ typedef enum {
   FA_ERR_WORKSPACE = 6    /* backward workspace missing or smaller than fa_bwd_workspace_size */
 } fa_status;
 
-/* Limits: d in {64, 96, 128, 256} (96 runs the d = 128 kernels on zero-filled columns; the
- * backward and the FP8 forward take d <= 128); B, H, N >= 1; B*H*N < 2^31;
- * B*H*ceil(N/256) < 2^31. */
+/* Limits: d in {64, 96, 128, 256} (96 runs the d = 128 kernels on zero-filled columns; the FP8
+ * forward takes d <= 128; d = 256 has no dropout); B, H, N >= 1; B*H*N < 2^31;
+ * B*H*ceil(N/256) < 2^31. At d = 256 the backward runs its main work in two passes over the
+ * key tiles (dV, then dK and dQ), because dK and dV of a 128-key tile fill all of TMEM. */
 
 /* Masks of the extended entry points. */
 typedef enum {
@@ -69,9 +70,8 @@ typedef enum {
  * uses key/value head h / (H / H_kv) (grouped heads; H_kv = 1 is a single shared K/V head),
  * and dk, dv of a key/value head sum over the query heads that share it. A query row that sees
  * no key (FA_MASK_CAUSAL_BOTTOM_RIGHT with N_q > N_kv) gets o = 0, lse = -inf and dq = 0.
- * Limits: d in {64, 96, 128, 256}; all sizes >= 1; B*H*N_q and B*H_kv*N_kv < 2^31. d = 256 is
- * supported by the forward only (no dropout): the backward and the FP8 forward return
- * FA_ERR_UNSUPPORTED for it, and fa_bwd_ex_workspace_size returns 0. */
+ * Limits: d in {64, 96, 128, 256}; all sizes >= 1; B*H*N_q and B*H_kv*N_kv < 2^31. At d = 256
+ * dropout and the FP8 forward return FA_ERR_UNSUPPORTED. */
 typedef struct {
   int B, H, H_kv, N_q, N_kv, d;
   float scale; /* finite, > 0; normally 1/sqrt(d) */
@@ -143,9 +143,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * All calls on a device share the one scratch array, which keeps the last call's contents (each
  * call rewrites what it reads before reading it): calls that overlap on the GPU (different
  * streams, or host threads, without ordering between them) race on it and must be serialised
- * by the caller. d = 256 is rejected with FA_ERR_UNSUPPORTED, as by fa_bwd. A timed-out
- * in-kernel wait (the hang guard) is recorded in a status word built into the library, which
- * fa_check_status reads and clears (it allocates nothing). */
+ * by the caller. A timed-out in-kernel wait (the hang guard) is recorded in a status word
+ * built into the library, which fa_check_status reads and clears (it allocates nothing). */
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                          const void* dO, const float* lse, void* dq, void* dk, void* dv, int B,
                          int H, int N, int d, float scale, int causal, void* stream);
@@ -198,12 +197,12 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_des
  * While enabled on the calling thread, every kernel the library launches is bracketed by a
  * pair of CUDA events recorded on its launch stream. fa_profile_read() waits for those events
  * and writes, per kernel kind k (0 = forward, 1 = backward preprocess, 2 = backward main,
- * 3 = backward dQ conversion, 4 = FP8 forward, 5 = FP8 V transpose, 6 = d = 256 forward;
- * FA_KERNEL_KINDS in total), the number of launches to
+ * 3 = backward dQ conversion, 4 = FP8 forward, 5 = FP8 V transpose, 6 = d = 256 forward,
+ * 7 = d = 256 backward dV pass, 8 = d = 256 backward dK/dQ pass; FA_KERNEL_KINDS in total), the number of launches to
  * launches[k] and their summed device time in milliseconds to ms[k], then forgets them.
  * n is the length of both arrays (>= FA_KERNEL_KINDS). Events are created by the library and
  * reused; no device memory is allocated. */
-#define FA_KERNEL_KINDS 7
+#define FA_KERNEL_KINDS 9
 fa_status fa_profile_enable(int on);
 fa_status fa_profile_read(double* ms, long long* launches, int n);
 /* Name of kernel kind k ("" if out of range). */

@@ -186,12 +186,20 @@ def test_debug_stall_hook_validation_without_gpu(lib):
     assert lib.fa_debug_stall_next(-1, 0, 0) == 0  # disarm
 
 
-def test_noalloc_rejects_d256_without_gpu(lib):
-    """No backward kernel exists at d = 256: fa_bwd_noalloc refuses it before any CUDA call, so
-    its scratch-size check never sees a size it was not written for."""
+def test_noalloc_d256_over_builtin_scratch_rejected_without_gpu(lib):
+    """At d = 256 the scratch fa_bwd_noalloc needs is sized like fa_bwd's workspace for d = 256
+    (fp32 dQ accumulator of 256 columns): sizes beyond the built-in 64 MiB are refused before any
+    CUDA call."""
+    B, H, N = 4, 16, 4096
+    assert fa.fa_bwd_workspace_size(B, H, N, 256) >= B * H * N * 256 * 4 > 64 << 20
     fake = 1 << 24
-    for B, H, N in ((1, 1, 128), (4, 16, 4096)):
-        st = lib.fa_bwd_noalloc(fake, fake * 2, fake * 3, fake * 4, fake * 5, fake * 6, fake * 7,
-                                fake * 8, fake * 9, B, H, N, 256, 0.0625, 1, None)
-        assert st == 2
-        assert "d <= 128" in fa.fa_last_error_string()
+    st = lib.fa_bwd_noalloc(fake, fake * 2, fake * 3, fake * 4, fake * 5, fake * 6, fake * 7,
+                            fake * 8, fake * 9, B, H, N, 256, 0.0625, 1, None)
+    assert st == 2
+    assert "built into the library" in fa.fa_last_error_string()
+
+
+def test_d256_backward_workspace_without_gpu(lib):
+    s = fa.FaAttnShape(2, 4, 2, 100, 300, 256, 0.0625, 1)
+    ws = lib.fa_bwd_ex_workspace_size(ctypes.byref(s))
+    assert ws == fa.fa_bwd_workspace_size(2, 4, 100, 256) > 2 * 4 * 100 * 256 * 4

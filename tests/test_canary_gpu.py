@@ -3,7 +3,7 @@ offer): every output and workspace of the library is placed inside a larger buff
 margins (8 KiB on each side) hold a sentinel byte pattern, and after the call every margin byte
 must be unchanged. The cases are the ones where the kernels clip: ragged row counts (TMA stores
 drop rows past N), d = 96 (stores drop columns 96..127), grouped heads, unequal lengths, rows
-that see no key, keys that no query sees, the d = 256 forward and the FP8 forward."""
+that see no key, keys that no query sees, the d = 256 forward and backward and the FP8 forward."""
 
 from __future__ import annotations
 
@@ -99,16 +99,27 @@ def test_forward_backward_write_only_their_outputs(case, dropout):
                                   (2, 4, 2, 513, 513, True), (1, 2, 1, 100, 700, "bottom_right"),
                                   (1, 2, 2, 700, 300, "bottom_right")],
                          ids=lambda c: "b%dh%dkv%dq%dk%d-%s" % c)
-def test_d256_forward_writes_only_its_outputs(case):
+def test_d256_forward_backward_write_only_their_outputs(case):
     B, H, H_kv, N_q, N_kv, mask = case
     x = make_inputs_ex(B, H, H_kv, N_q, N_kv, 256, seed=950 + N_q + N_kv)
-    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
     o = Guarded((B, H, N_q, 256), torch.bfloat16)
     lse = Guarded((B, H, N_q), torch.float32)
     fa.fa_fwd_ex(q, k, v, o.t, lse.t, causal=mask)
     fa.fa_check_status()
     o.check("o")
     lse.check("lse")
+    dq = Guarded((B, H, N_q, 256), torch.bfloat16)
+    dk = Guarded((B, H_kv, N_kv, 256), torch.bfloat16)
+    dv = Guarded((B, H_kv, N_kv, 256), torch.bfloat16)
+    ws = Guarded(None, torch.uint8,
+                 nbytes=fa.fa_bwd_ex_workspace_size(B, H, H_kv, N_q, N_kv, 256, mask))
+    fa.fa_bwd_ex(q, k, v, o.t, do, lse.t, dq.t, dk.t, dv.t, ws.t, causal=mask)
+    fa.fa_check_status()
+    for g, n in ((dq, "dq"), (dk, "dk"), (dv, "dv"), (ws, "workspace")):
+        g.check(n)
+    for t in (dq.t, dk.t, dv.t):
+        assert torch.isfinite(t).all()
 
 
 @pytest.mark.parametrize("case", [(1, 1, 1, 1, 1, 64, False), (1, 2, 2, 300, 300, 128, True),

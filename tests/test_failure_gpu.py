@@ -70,11 +70,11 @@ def test_forward_kernel_timeout_unwinds(d, causal, skip):
 
 
 @pytest.mark.parametrize("d,causal,skip", [(128, True, 0), (128, False, 1), (64, True, 0),
-                                           (64, False, 2)])
+                                           (64, False, 2), (256, True, 0), (256, False, 1)])
 def test_backward_kernel_timeout_unwinds(d, causal, skip):
-    """The backward main kernel (the 128-row kernel at d = 128, the 64-row one at d = 64): a query
-    tile never arrives; the call reports FA_ERR_TIMEOUT, and the next backward on the same
-    context matches the oracle."""
+    """The backward main kernel (the 128-row kernel at d = 128, the 64-row one at d = 64, the dV
+    pass at d = 256): a query tile never arrives; the call reports FA_ERR_TIMEOUT, and the next
+    backward on the same context matches the oracle."""
     fa.fa_check_status()
     x = make_inputs(1, 2, 384, d, seed=50 + d + skip)
     q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))

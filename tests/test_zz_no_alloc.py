@@ -56,12 +56,21 @@ def test_noalloc_rejects_sizes_beyond_builtin_scratch():
     assert "built into the library" in fa.fa_last_error_string()
 
 
-def test_noalloc_rejects_d256_before_any_launch():
-    """d = 256 has no backward kernel: the call is refused with FA_ERR_UNSUPPORTED before the
-    scratch-size check and before any launch (the pointers are never touched)."""
-    fake = 1 << 24
-    for B, H, N in ((1, 1, 128), (4, 16, 4096)):
-        st = fa.lib().fa_bwd_noalloc(fake, fake * 2, fake * 3, fake * 4, fake * 5, fake * 6,
-                                     fake * 7, fake * 8, fake * 9, B, H, N, 256, 0.0625, 1, None)
-        assert st == 2
-        assert "d <= 128" in fa.fa_last_error_string()
+def test_noalloc_d256_matches_fa_bwd():
+    """d = 256 (the two-pass backward) through the built-in scratch: same gradients as fa_bwd."""
+    B, H, N, d = 1, 2, 700, 256
+    x = make_inputs(B, H, N, d, seed=39)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_forward(q, k, v, causal=True)
+    ref = fa.attention_backward(q, k, v, o, do, lse, causal=True)
+    fa.fa_check_status()
+    for call in range(2):
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        for t in (dq, dk, dv):
+            t.fill_(float("nan"))
+        fa.fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal=True)
+        fa.fa_check_status()
+        for g, r, n in zip((dq, dk, dv), ref, ("dQ", "dK", "dV")):
+            assert torch.isfinite(g).all(), f"call {call}: {n} not fully written"
+            assert grad_rel_error(g, to64(r)) <= TOL_GRAD_REL, f"call {call}: {n}"
+        assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
