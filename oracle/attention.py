@@ -314,13 +314,17 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, do=None, dropout=N
 
 
 def attention_keys(q, k, v, do, scale: float, causal, head, keys, block_rows: int = 512,
-                   dropout=None):
+                   dropout=None, stats=None):
     """dK and dV rows for selected keys j of one key/value head (leading index tuple `head`,
     e.g. (b, h_kv)).
 
     dV_j = sum_i P_ij dO_i and dK_j = scale sum_i dS_ij q_i over the query rows that see key j,
     in every query head that uses this key/value head. Needs lse_i and D_i of those rows, so
-    their full forward is computed first. Returns (dK_rows [n, d], dV_rows [n, d]).
+    their full forward is computed first, unless `stats` = (O [n, d], lse [n]) of the query
+    head's rows is given (one query head per key/value head only; only the rows that see the
+    selected keys are read, so the others may hold anything, e.g. NaN). This lets a caller take
+    those rows from ``attention_rows`` when the full forward is too long to run.
+    Returns (dK_rows [n, d], dV_rows [n, d]).
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     mode = _mode(causal)
@@ -337,11 +341,17 @@ def attention_keys(q, k, v, do, scale: float, causal, head, keys, block_rows: in
     off = (nk - n) if mode == "bottom_right" else 0
     dk_out = np.zeros((len(keys), kh.shape[1]))
     dv_out = np.zeros((len(keys), vh.shape[1]))
+    if stats is not None and len(q_heads) != 1:
+        raise ValueError("stats is supported with one query head per key/value head")
     for qh_idx in q_heads:
         qh, doh = q[qh_idx], do[qh_idx]
         bh = _flat_head(qh_idx, q.shape)
-        o, lse = _forward_one_head(qh, kh, vh, scale, mode, block_rows, bh, drop)
-        dd = np.sum(doh * o, axis=1)
+        if stats is None:
+            o, lse = _forward_one_head(qh, kh, vh, scale, mode, block_rows, bh, drop)
+        else:
+            o, lse = _f64(stats[0]), _f64(stats[1])
+        with np.errstate(invalid="ignore"):  # rows outside i0 .. n may hold NaN
+            dd = np.sum(doh * o, axis=1)
         for t, j in enumerate(int(x) for x in keys):
             i0 = 0 if mode == "none" else max(0, j - off)  # rows i with j <= i + off see key j
             if i0 >= n:

@@ -215,3 +215,21 @@ def test_mutants_of_extended_cases_are_caught(kind):
     ref = _torch_ref(q, k, v, do, 0.5, "bottom_right")[0]
     assert np.max(np.abs(_mutant_forward("none")(q, k, v, 0.5, "bottom_right") - ref)) < 1e-12
     assert np.max(np.abs(_mutant_forward(kind)(q, k, v, 0.5, "bottom_right") - ref)) > 1e-3
+
+
+def test_attention_keys_with_given_row_stats():
+    """attention_keys with the rows' (O, lse) given reproduces the version that computes the
+    forward itself; rows that do not see the selected keys are not read (NaN there is fine)."""
+    rng = np.random.default_rng(11)
+    B, H, N, d = 1, 2, 40, 8
+    q, k, v, do = (rng.standard_normal((B, H, N, d)) for _ in range(4))
+    scale = 0.3
+    keys = [25, 31, 39]
+    for h in range(H):
+        ref = attention_keys(q, k, v, do, scale, True, (0, h), keys)
+        o, lse = attention_forward(q[0, h], k[0, h], v[0, h], scale, True)
+        o_s, lse_s = o.copy(), lse.copy()
+        o_s[:25], lse_s[:25] = np.nan, np.nan  # causal: key 25 is seen by rows 25 .. N-1 only
+        got = attention_keys(q, k, v, do, scale, True, (0, h), keys, stats=(o_s, lse_s))
+        for a, b in zip(got, ref):
+            assert np.abs(a - b).max() <= 1e-12 * np.abs(b).max()
