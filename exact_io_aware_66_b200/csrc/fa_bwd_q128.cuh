@@ -260,7 +260,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int t = 0; t < 4; ++t)
           *reinterpret_cast<uint4*>(dsb + sw128_offset(r, 4 * h + t)) =
               make_uint4(dsk[4 * t], dsk[4 * t + 1], dsk[4 * t + 2], dsk[4 * t + 3]);
+        // and to TMEM over this warpgroup's first dP^T columns, already read (h = 0 writes
+        // columns 64w .. 64w+15, below the ones h = 1 reads): the A operand of dK
+        tmem_st_32x32b_x16(tmem + L::tDP + 64 * w + 16 * h + lane_off, dsk);
       }
+      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(L::bDSDone));
@@ -367,7 +371,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dDO_k = sdesc_sw128(sbase + L::kDO, 16, 1024);        // dO, K-major
       const uint64_t dQ_mn = sdesc_sw128(sbase + L::kQ, L::kBox, 1024);    // Q, MN-major
       const uint64_t dDO_mn = sdesc_sw128(sbase + L::kDO, L::kBox, 1024);  // dO, MN-major
-      const uint64_t dDS_k = sdesc_sw128(sbase + L::kDS, 16, 1024);        // dS^T, K-major
       const uint64_t dDS_mn = sdesc_sw128(sbase + L::kDS, L::kBox, 1024);  // dS^T, MN-major
       // K-step kk of a K-major operand: box kk / 4, 32 bytes per step inside the 128-byte row;
       // of an MN-major operand: 16 rows of 128 bytes.
@@ -391,11 +394,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           umma_ts(tmem + L::tDV, tmem + L::tS + (kk >> 2) * 64 + (kk & 3) * 8,
                   sdesc_advance(dDO_mn, kk * 2048), id_acc, (kk > 0 || i > 0) ? 1u : 0u);
       };
-      auto mma_dk = [&](int i) {  // dK += dS^T Q
+      auto mma_dk = [&](int i) {  // dK += dS^T Q; dS^T from TMEM (its bf16 copy over dP^T)
         const uint32_t so = static_cast<uint32_t>(i & 1) * L::kTile;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + L::tDK, sdesc_advance(dDS_k, kmaj(kk)),
+          umma_ts(tmem + L::tDK, tmem + L::tDP + (kk >> 2) * 64 + (kk & 3) * 8,
                   sdesc_advance(dQ_mn, so + kk * 2048), id_acc, (kk > 0 || i > 0) ? 1u : 0u);
       };
       auto mma_dq = [&]() {  // dQ^T = K^T dS^T, into the dP^T columns
