@@ -847,7 +847,7 @@ fa_status launch_fwd_fp8(DeviceState* ds, const void* q8, const void* k8, const 
   if ((st = make_bf16_map(&to, o, s.d, s.N_q, BH, 32)) != FA_OK) return st;
 
   {
-    const dim3 grid((s.N_kv + 63) / 64, (s.d + 63) / 64, BHkv);
+    const dim3 grid((s.N_kv + fa::kTrKeys - 1) / fa::kTrKeys, (s.d + 63) / 64, BHkv);
     if (grid.z > 65535) return set_err(FA_ERR_UNSUPPORTED, "B*H_kv > 65535 for the fp8 path");
     ProfileScope prof(5, stream);
     fa::fa_fp8_transpose_v<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(v8), vt, s.N_kv,

@@ -436,30 +436,50 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
-// V [rows][d] (E4M3 bytes) -> V^T [d][ld] per head, 64 x 64-byte tiles through shared memory.
-// Grid: (ceil(N_kv / 64), ceil(d / 64), B * H_kv), 256 threads; d a multiple of 16.
+// V [rows][d] (E4M3 bytes) -> V^T [d][ld] per head. A block transposes 128 keys x 64 columns:
+// each thread loads 4 x 4-byte blocks (four 32-bit words from rows r .. r+3), turns them into
+// the four columns' words with byte permutes, and writes those to shared memory; the block then
+// stores rows of 128 transposed keys with 16-byte stores. (Byte-wide shared-memory accesses,
+// one per element, made an earlier version several times slower than a copy.)
+// Grid: (ceil(N_kv / 128), ceil(d / 64), B * H_kv), 256 threads; d a multiple of 16.
+constexpr int kTrKeys = 128;
 __global__ void __launch_bounds__(256)
     fa_fp8_transpose_v(const uint8_t* __restrict__ v, uint8_t* __restrict__ vt, int N_kv, int d,
                        int ld) {
-  __shared__ uint8_t tile[64][64 + 4];
-  const int k0 = blockIdx.x * 64, c0 = blockIdx.y * 64;
+  // T[c][k / 4]: column c (0..63) of the tile, keys as bytes; rows of 128 keys padded to 144 bytes
+  __shared__ __align__(16) uint32_t T[64][36];
+  const int k0 = blockIdx.x * kTrKeys, c0 = blockIdx.y * 64;
   const size_t head = blockIdx.z;
-  const int r = threadIdx.x >> 2, part = (threadIdx.x & 3) * 16;
-  {
-    uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (k0 + r < N_kv && c0 + part < d)  // d is a multiple of 16
-      x = *reinterpret_cast<const uint4*>(v + (head * N_kv + k0 + r) * d + c0 + part);
-    const uint8_t* b = reinterpret_cast<const uint8_t*>(&x);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) tile[r][part + i] = b[i];
+  for (int rep = 0; rep < 2; ++rep) {
+    // 4 x 4 block number (512 per tile): a warp covers 8 row groups x 4 column groups
+    const int b = threadIdx.x + 256 * rep;
+    const int rg = (b & 7) | (((b >> 5) & 3) << 3);  // 0 .. 31: keys 4 rg .. 4 rg + 3
+    const int cg = ((b >> 3) & 3) | ((b >> 7) << 2);  // 0 .. 15: columns 4 cg .. 4 cg + 3
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      w[i] = 0u;
+      if (k0 + 4 * rg + i < N_kv && c0 + 4 * cg < d)  // d % 16 == 0: the whole word is inside
+        w[i] = *reinterpret_cast<const uint32_t*>(v + (head * N_kv + k0 + 4 * rg + i) * d + c0 +
+                                                  4 * cg);
+    }
+    // byte j of word i is element (key 4 rg + i, column 4 cg + j); gather each column's bytes
+    const uint32_t t0 = __byte_perm(w[0], w[1], 0x5140), t1 = __byte_perm(w[0], w[1], 0x7362);
+    const uint32_t t2 = __byte_perm(w[2], w[3], 0x5140), t3 = __byte_perm(w[2], w[3], 0x7362);
+    T[4 * cg + 0][rg] = __byte_perm(t0, t2, 0x5410);
+    T[4 * cg + 1][rg] = __byte_perm(t0, t2, 0x7632);
+    T[4 * cg + 2][rg] = __byte_perm(t1, t3, 0x5410);
+    T[4 * cg + 3][rg] = __byte_perm(t1, t3, 0x7632);
   }
   __syncthreads();
-  if (k0 + part < N_kv && c0 + r < d) {  // 16 keys starting inside the row (ld % 16 == 0)
-    uint4 y;
-    uint8_t* b = reinterpret_cast<uint8_t*>(&y);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) b[i] = tile[part + i][r];
-    *reinterpret_cast<uint4*>(vt + (head * d + c0 + r) * static_cast<size_t>(ld) + k0 + part) = y;
+  for (int rep = 0; rep < 2; ++rep) {
+    const int e = threadIdx.x + 256 * rep;  // 16-byte chunk: 64 columns x 8 chunks of keys
+    const int c = e >> 3, part = (e & 7) * 16;
+    if (c0 + c < d && k0 + part < N_kv)  // ld % 16 == 0: the chunk fits in the row
+      *reinterpret_cast<uint4*>(vt + (head * d + c0 + c) * static_cast<size_t>(ld) + k0 + part) =
+          *reinterpret_cast<const uint4*>(&T[c][part / 4]);
   }
 }
 
