@@ -66,6 +66,9 @@ WORKLOADS = {
                                              True, 4, True, row_samples=512, key_samples=64),
     "causal_fwd_b1h8n131072d128": Workload("causal_fwd_b1h8n131072d128", 1, 8, 131072, 128, True,
                                            5, False, spike_every=97, spike=8.0, row_samples=256),
+    # head dimension 96 (run by the d = 128 kernels on zero-filled columns), for measurement
+    "causal_train_b4h16n4096d96": Workload("causal_train_b4h16n4096d96", 4, 16, 4096, 96, True, 7,
+                                           True, mult=0.5, row_samples=256, key_samples=64),
     # head dimension 256, for measurement
     "causal_fwd_b2h16n8192d256": Workload("causal_fwd_b2h16n8192d256", 2, 16, 8192, 256, True, 6,
                                           False, row_samples=256),

@@ -63,10 +63,12 @@ def test_fwd_bwd_full_size_every_element(name):
               f"mean-abs {float(np.abs(to64(g) - r).mean()):.3e}")
 
 
-def test_bwd_long_sequence_sampled():
-    """B=1, H=16, N=16384, d=128 causal: dQ on 512 sampled rows, dK and dV on 64 sampled keys
-    (drawn from 2 seeded heads, whose full forward the oracle needs)."""
-    w = WORKLOADS["causal_train_b1h16n16384d128"]
+@pytest.mark.parametrize("name", ["causal_train_b1h16n16384d128", "causal_train_b4h16n4096d96"])
+def test_bwd_long_sequence_sampled(name):
+    """B=1, H=16, N=16384, d=128 causal (and the d = 96 measurement workload, B4 H16 N4096):
+    dQ on the sampled rows, dK and dV on 64 sampled keys (drawn from 2 seeded heads, whose full
+    forward the oracle needs)."""
+    w = WORKLOADS[name]
     x = workload_inputs(w)
     _, _, dq, dk, dv = _fwd_bwd(x, w.causal)
     q, k, v, do = (x[n].float().numpy() for n in ("q", "k", "v", "do"))
