@@ -116,7 +116,7 @@ struct DeviceState {
   std::atomic<bool> fp8_attr[2] = {};  // [causal]
   std::atomic<bool> d256_attr[2] = {};  // [causal]
   std::atomic<bool> bwd_attr[2][2][2] = {};
-  std::atomic<bool> bwd128_attr[2] = {};  // [causal]
+  std::atomic<bool> bwd128_attr[4] = {};  // [2 (d = 128) + causal]
   std::atomic<bool> bwd256_attr[2] = {};  // [causal]
 };
 std::mutex g_mu;
@@ -430,15 +430,15 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   return FA_OK;
 }
 
-// Backward at d = 128 (and 96) without dropout: the 128-row query tile kernel
+// Backward at d = 64 and d = 128 (and 96) without dropout: the 128-row query tile kernel
 // (fa_bwd_q128.cuh), between the same preprocess and dQ conversion as launch_bwd.
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 fa_status launch_bwd_q128(DeviceState* ds, const void* q, const void* k, const void* v,
                           const void* o, const void* dO, const float* lse, void* dq, void* dk,
                           void* dv, void* workspace, const Shape& s, cudaStream_t stream) {
-  using L = fa::Bwd128Layout;
-  auto kern = fa::fa_bwd_main_q128<CAUSAL>;
-  std::atomic<bool>& attr = ds->bwd128_attr[CAUSAL];
+  using L = fa::Bwd128Layout<D>;
+  auto kern = fa::fa_bwd_main_q128<D, CAUSAL>;
+  std::atomic<bool>& attr = ds->bwd128_attr[(D == 128 ? 2 : 0) + CAUSAL];
   if (!attr) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
@@ -477,12 +477,14 @@ fa_status launch_bwd_q128(DeviceState* ds, const void* q, const void* k, const v
   if ((st = make_map(&tD, Dvec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, BH, 1, 128, 1,
                      CU_TENSOR_MAP_SWIZZLE_NONE, n64)) != FA_OK)
     return st;
-  // dQ accumulator: fp32 [BH][N_q][d], reduction boxes of 32 columns x 64 rows
-  if ((st = make_map(&tacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, s.d, N, BH, 32, 64,
-                     CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
+  // dQ accumulator: fp32 [BH][N_q][d], reduction boxes of 32 columns x 64 rows; at d = 64,
+  // 32 x 32 boxes in the 128-byte swizzled layout (the drain writes query rows)
+  if ((st = make_map(&tacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, s.d, N, BH, 32,
+                     D == 64 ? 32 : 64,
+                     D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE)) != FA_OK)
     return st;
 
-  const long long prep_threads = rows * 16;
+  const long long prep_threads = rows * (D == 64 ? 8 : 16);
   const long long prep_blocks = (prep_threads + fa::kPrepThreads - 1) / fa::kPrepThreads;
   if (prep_blocks >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
   {
@@ -494,8 +496,8 @@ fa_status launch_bwd_q128(DeviceState* ds, const void* q, const void* k, const v
       fa::fa_bwd_preprocess<96><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc, Dvec,
                                                                      lse2, rows, N, n64);
     else
-      fa::fa_bwd_preprocess<128><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc,
-                                                                      Dvec, lse2, rows, N, n64);
+      fa::fa_bwd_preprocess<D><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc,
+                                                                    Dvec, lse2, rows, N, n64);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd preprocess launch");
@@ -724,10 +726,7 @@ fa_status bwd_dispatch_d(DeviceState* ds, const void* q, const void* k, const vo
                          void* dv, void* workspace, const Shape& s, cudaStream_t stream) {
   if (s.dropout)
     return launch_bwd<D, CAUSAL, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
-  if constexpr (D == 128)
-    return launch_bwd_q128<CAUSAL>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
-  else
-    return launch_bwd<D, CAUSAL, false>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
+  return launch_bwd_q128<D, CAUSAL>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
 }
 
 fa_status bwd_dispatch(DeviceState* ds, const void* q, const void* k, const void* v, const void* o,
@@ -952,7 +951,7 @@ struct NoAllocDevice {
   void* scratch = nullptr;  // device address of g_noalloc_scratch on this device
   int* status = nullptr;    // device address of g_noalloc_status on this device
   bool bwd_attr[2][2][2] = {};
-  bool bwd128_attr[2] = {};
+  bool bwd128_attr[4] = {};
   bool bwd256_attr[2] = {};
 };
 
@@ -1140,10 +1139,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
     local.status = nd.status;
     local.checked = local.is_sm100 = true;
     copy_flags(local.bwd_attr, nd.bwd_attr);
-    for (int c = 0; c < 2; ++c) {
-      local.bwd128_attr[c].store(nd.bwd128_attr[c]);
-      local.bwd256_attr[c].store(nd.bwd256_attr[c]);
-    }
+    for (int c = 0; c < 4; ++c) local.bwd128_attr[c].store(nd.bwd128_attr[c]);
+    for (int c = 0; c < 2; ++c) local.bwd256_attr[c].store(nd.bwd256_attr[c]);
   }
   // The first kernel of the backward rewrites every scratch byte the later ones read (dQ
   // accumulator zeroed, D and -lse*log2e recomputed), so the previous call's contents do not
@@ -1153,10 +1150,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   {
     std::lock_guard<std::mutex> lock(g_mu);
     copy_flags(g_noalloc[dev].bwd_attr, local.bwd_attr);
-    for (int c = 0; c < 2; ++c) {
-      g_noalloc[dev].bwd128_attr[c] = local.bwd128_attr[c].load();
-      g_noalloc[dev].bwd256_attr[c] = local.bwd256_attr[c].load();
-    }
+    for (int c = 0; c < 4; ++c) g_noalloc[dev].bwd128_attr[c] = local.bwd128_attr[c].load();
+    for (int c = 0; c < 2; ++c) g_noalloc[dev].bwd256_attr[c] = local.bwd256_attr[c].load();
   }
   return st;
 }

@@ -1,5 +1,5 @@
-// fa_bwd_q128.cuh — exact attention backward for sm_100a with 128-row query tiles (d = 128,
-// and d = 96 through zero-filled columns; no dropout).
+// fa_bwd_q128.cuh — exact attention backward for sm_100a with 128-row query tiles (d = 64 and
+// d = 128, and d = 96 through zero-filled columns; no dropout).
 //
 // Same mathematics as fa_bwd_main (fa_bwd.cuh): with P = exp(S - lse),
 //     dV = P^T dO,  dP = dO V^T,  D_i = dO_i . O_i,  dS = P o (dP - D),
@@ -12,7 +12,8 @@
 //     every tcgen05 product is M = 128, N = 128 (an N = 64 product reads 6 KB of shared-memory
 //     operands per k-step for half the work of an N = 128 one, which reads 8 KB).
 //   * TMEM holds exactly four 128-column fp32 regions: dV, dK, S^T (then P^T in place) and dP^T
-//     (then dQ^T in place). Nothing is double buffered; instead the MMA issue order is
+//     (then dQ^T in place; at d = 64, dQ = dS K with the queries on the lanes, since an M = 64
+//     product would leave half the lanes idle). Nothing is double buffered; the MMA issue order is
 //         S(i), dK(i-1), dQ(i-1), dV(i), dP(i), S(i+1), ...
 //     so the elementwise warps turn S^T(i) into P^T(i) while the tensor core finishes tile i-1,
 //     and the dQ^T(i-1) drain overlaps dV(i).
@@ -23,8 +24,9 @@
 //     single slot, refilled after dP(i), its last reader, and needed again by dV(i+1) three
 //     products later. That single slot is what pays for the staging buffer.
 //
-// Shared memory (about 227 KB): K, V (32 KB each), two Q stages (64 KB), dO (32 KB), dS^T
-// (32 KB), dQ staging (32 KB), two stages of per-row terms (2 KB), barriers. The 128-byte
+// Shared memory at d = 128 (about 227 KB): K, V (32 KB each), two Q stages (64 KB), dO (32 KB),
+// dS^T (32 KB), dQ staging (32 KB), two stages of per-row terms (2 KB), barriers; at d = 64 the
+// five 128 x d tiles take half as much (163 KB in all). The 128-byte
 // swizzle needs a 1024-byte aligned base; a misaligned base is reported through the status word
 // (code 7) instead of being used.
 #pragma once
@@ -32,16 +34,18 @@
 
 namespace fa {
 
+template <int D>
 struct Bwd128Layout {
   static constexpr int kBox = 128 * 64 * 2;        // TMA box: 128 rows x 64 bf16 columns (SW128)
-  static constexpr int kTile = 2 * kBox;           // 128 rows x 128 columns
+  static constexpr int kBoxes = D / 64;            // boxes per 128-row tile
+  static constexpr int kTile = kBoxes * kBox;      // 128 rows x D columns
   static constexpr int kK = 0;
   static constexpr int kV = kTile;
   static constexpr int kQ = 2 * kTile;             // + stage * kTile (2 stages)
   static constexpr int kDO = 4 * kTile;            // one slot
   static constexpr int kDS = 5 * kTile;            // dS^T [128 keys][128 queries], two 64-query boxes
-  static constexpr int kDQ = 6 * kTile;            // dQ staging: 4 warps x (64 rows x 32 fp32)
-  static constexpr int kRow = 7 * kTile;           // per Q stage (1 KB): lse2[128], then D[128]
+  static constexpr int kDQ = kDS + 2 * kBox;       // dQ staging, 32 KB (4 warps x 8 KB)
+  static constexpr int kRow = kDQ + 2 * kBox;      // per Q stage (1 KB): lse2[128], then D[128]
   static constexpr int kBars = kRow + 2 * 1024;
 
   static constexpr int bKV = 0;
@@ -66,7 +70,8 @@ struct Bwd128Layout {
   // TMEM columns
   static constexpr uint32_t tDV = 0, tDK = 128, tS = 256, tDP = 384;
 };
-static_assert(Bwd128Layout::kBytes <= 227 * 1024, "q128 backward shared memory");
+static_assert(Bwd128Layout<128>::kBytes <= 227 * 1024, "q128 backward shared memory");
+static_assert(Bwd128Layout<64>::kBytes <= 227 * 1024, "q128 backward shared memory");
 
 // Register split (setmaxnreg, per warpgroup): the drain warpgroup holds its lanes' 128 dQ^T
 // columns in registers while it stages them; the two elementwise warpgroups (64 fp32
@@ -88,7 +93,7 @@ __device__ __forceinline__ void bwd128_setmaxnreg() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(R));
 }
 
-template <bool CAUSAL>
+template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_q128(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
@@ -99,7 +104,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                      const __grid_constant__ CUtensorMap tmDQacc,
                      const __grid_constant__ CUtensorMap tmDK,
                      const __grid_constant__ CUtensorMap tmDV, const BwdParams p) {
-  using L = Bwd128Layout;
+  using L = Bwd128Layout<D>;
   using R = Bwd128Regs;
   // No static shared memory in this kernel, so the dynamic block starts at the beginning of
   // the CTA's shared window. The layout uses all of it (no slack to realign), so the 1024-byte
@@ -279,7 +284,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int region = L::kQ + w * L::kTile;
       uint8_t* stage = gbase + region;
 #pragma unroll
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; c < D; c += 32) {
         uint32_t v[32];
         if (n_i > 0) {
           tmem_ld_32x32b_x32(tmem + tcol + c + lane_off, v);
@@ -305,7 +310,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (lane == 0) {
         const CUtensorMap* map = w == 0 ? &tmDV : &tmDK;
 #pragma unroll
-        for (int bx = 0; bx < 2; ++bx)
+        for (int bx = 0; bx < L::kBoxes; ++bx)
           tma_store_3d(map, sbase + region + bx * L::kBox + (warp & 3) * 4096, 64 * bx,
                        k0 + (warp & 3) * 32, bh);
         bulk_commit_group();
@@ -314,8 +319,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     } else if (ok) {
       fail(p.status, abort_flag, 5);
     }
+  } else if (warp < 12 && D == 64) {
+    // ------------------------------------------------------- dQ drain (d = 64) ----------
+    // dQ(i) sits in TMEM as [128 queries (lanes)][64 columns]: warp wq holds queries
+    // [32 wq, 32 wq + 32) of the tile and stages them as two 32 x 32 fp32 boxes in the 128-byte
+    // swizzled layout (16-byte stores, conflict-free), each added into the accumulator by one
+    // TMA reduction.
+    bwd128_setmaxnreg<R::kDrain>();
+    const int wq = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const float scale = p.scale;
+    uint8_t* stageb = gbase + L::kDQ + wq * 8192;
+    const uint32_t stage_s = sbase + L::kDQ + wq * 8192;
+    bool ok = true;
+    for (int i = 0; i < n_i; ++i) {
+      if (!warp_wait(bar(L::bDQFull), i & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t v[64];
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        tmem_ld_32x32b_x32(tmem + L::tDP + 32 * c + lane_off,
+                           *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+      tmem_ld_wait();
+      reg_fence(v);
+      tc_fence_before();
+      mbar_arrive(bar(L::bDQFree));
+      const int q0 = 128 * q_tile(i) + 32 * wq, qh = q_head(i);
+      if (q0 >= p.N) continue;  // no rows of this warp's slice exist
+      if (lane == 0) bulk_wait_group_read0();  // the previous reduction has read the staging
+      __syncwarp();
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          *reinterpret_cast<float4*>(stageb + b * 4096 + sw128_offset(lane, t)) =
+              make_float4(__uint_as_float(v[32 * b + 4 * t]) * scale,
+                          __uint_as_float(v[32 * b + 4 * t + 1]) * scale,
+                          __uint_as_float(v[32 * b + 4 * t + 2]) * scale,
+                          __uint_as_float(v[32 * b + 4 * t + 3]) * scale);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_3d(&tmDQacc, stage_s, 0, q0, qh);
+        tma_reduce_add_3d(&tmDQacc, stage_s + 4096, 32, q0, qh);
+        bulk_commit_group();
+      }
+    }
+    if (!ok) fail(p.status, abort_flag, 5);
+    if (lane == 0) bulk_wait_group0();
   } else if (warp < 12) {
-    // ---------------------------------------------------------------- dQ drain ----------
+    // ------------------------------------------------------ dQ drain (d = 128) ----------
     bwd128_setmaxnreg<R::kDrain>();
     const int wq = warp & 3;                        // dQ^T rows (d) [32 wq, 32 wq + 32)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -362,8 +415,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (warp == 12 && lane == 0) {
       // ------------------------------------------------------------------- MMA ----------
       const uint32_t id_s = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
-      const uint32_t id_acc = idesc_bf16_f32(128, 128, false, true); // dV, dK
-      const uint32_t id_dq = idesc_bf16_f32(128, 128, true, true);   // dQ^T
+      const uint32_t id_acc = idesc_bf16_f32(128, D, false, true);   // dV, dK
+      const uint32_t id_dq = idesc_bf16_f32(128, 128 * D / 128, true, true);  // dQ^T, or dQ
       const uint64_t dK_k = sdesc_sw128(sbase + L::kK, 16, 1024);          // K, K-major
       const uint64_t dV_k = sdesc_sw128(sbase + L::kV, 16, 1024);          // V, K-major
       const uint64_t dKt_mn = sdesc_sw128(sbase + L::kK, L::kBox, 1024);   // K^T, MN-major
@@ -378,13 +431,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       auto mma_s = [&](int i) {  // S^T = K Q^T
         const uint32_t so = static_cast<uint32_t>(i & 1) * L::kTile;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < D / 16; ++kk)
           umma_ss(tmem + L::tS, sdesc_advance(dK_k, kmaj(kk)), sdesc_advance(dQ_k, so + kmaj(kk)),
                   id_s, kk > 0 ? 1u : 0u);
       };
       auto mma_dp = [&]() {  // dP^T = V dO^T
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < D / 16; ++kk)
           umma_ss(tmem + L::tDP, sdesc_advance(dV_k, kmaj(kk)), sdesc_advance(dDO_k, kmaj(kk)),
                   id_s, kk > 0 ? 1u : 0u);
       };
@@ -401,11 +454,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           umma_ts(tmem + L::tDK, tmem + L::tDP + (kk >> 2) * 64 + (kk & 3) * 8,
                   sdesc_advance(dQ_mn, so + kk * 2048), id_acc, (kk > 0 || i > 0) ? 1u : 0u);
       };
-      auto mma_dq = [&]() {  // dQ^T = K^T dS^T, into the dP^T columns
+      auto mma_dq = [&]() {  // into the dP^T columns
+        if constexpr (D == 128) {  // dQ^T = K^T dS^T: M = d
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + L::tDP, sdesc_advance(dKt_mn, kk * 2048),
-                  sdesc_advance(dDS_mn, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tmem + L::tDP, sdesc_advance(dKt_mn, kk * 2048),
+                    sdesc_advance(dDS_mn, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
+        } else {  // dQ = dS K: M = 128 queries (dS^T read MN-major), N = d = 64 (K, MN-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tmem + L::tDP, sdesc_advance(dDS_mn, kk * 2048),
+                    sdesc_advance(dKt_mn, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
+        }
       };
       const uint64_t lim = p.limit_ns;
       bool ok = n_i == 0 || mbar_wait(bar(L::bKV), 0, abort_flag, lim);
@@ -453,7 +513,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (n_i > 0) {
         mbar_arrive_expect_tx(bar(L::bKV), 2 * L::kTile);
 #pragma unroll
-        for (int bx = 0; bx < 2; ++bx) {
+        for (int bx = 0; bx < L::kBoxes; ++bx) {
           tma_load_3d(sbase + L::kK + bx * L::kBox, &tmK, bar(L::bKV), 64 * bx, k0, bh);
           tma_load_3d(sbase + L::kV + bx * L::kBox, &tmV, bar(L::bKV), 64 * bx, k0, bh);
         }
@@ -471,7 +531,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (i != p.dbg_skip) {  // (the test hook leaves this tile out)
           mbar_arrive_expect_tx(bar(L::bQFull + st), L::kTile + 1024);
 #pragma unroll
-          for (int bx = 0; bx < 2; ++bx)
+          for (int bx = 0; bx < L::kBoxes; ++bx)
             tma_load_3d(sbase + L::kQ + so + bx * L::kBox, &tmQ, bar(L::bQFull + st), 64 * bx,
                         q0, qh);
           tma_load_3d(sbase + L::kRow + st * 1024, &tmLse2, bar(L::bQFull + st), q0, qh, 0);
@@ -485,7 +545,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mbar_arrive_expect_tx(bar(L::bOFull), L::kTile);
 #pragma unroll
-        for (int bx = 0; bx < 2; ++bx)
+        for (int bx = 0; bx < L::kBoxes; ++bx)
           tma_load_3d(sbase + L::kDO + bx * L::kBox, &tmDO, bar(L::bOFull), 64 * bx, q0, qh);
         issued_o = i + 1;
       }
