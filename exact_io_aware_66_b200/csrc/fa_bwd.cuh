@@ -200,12 +200,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // and dQ accumulator fit in L2; within a group the key tiles with the most query tiles
   // (causal) come first, cycling over the group's heads (longest-processing-time order).
   constexpr int QS = L::kQStages;
-  const int per_group = p.group * p.n_kv;
-  const int g0 = static_cast<int>(blockIdx.x / per_group) * p.group;
-  const int r_in = static_cast<int>(blockIdx.x % per_group);
-  const int gcur = min(p.group, p.BH_kv - g0);
-  const int j = r_in / gcur;
-  const int bh = g0 + r_in % gcur;  // key/value head
+  int j, bh;  // key tile, key/value head
+  grouped_unit(static_cast<int>(blockIdx.x), p.n_kv, p.BH_kv, p.group, j, bh);
   const int k0 = 128 * j;
   // First 64-row query tile with a query that sees a key of this tile (j <= i + off), and the
   // iterations: every query head that shares this key/value head, times its query tiles.

@@ -86,12 +86,8 @@ static_assert(Bwd256DkdqLayout::kAlloc + 16 <= 227 * 1024, "d = 256 dK/dQ pass s
 struct Bwd256Unit {
   int bh, k0, qi0, n_qt, n_i, qgroup;
   __device__ Bwd256Unit(const BwdParams& p, bool causal) {
-    const int per_group = p.group * p.n_kv;
-    const int g0 = static_cast<int>(blockIdx.x / per_group) * p.group;
-    const int r_in = static_cast<int>(blockIdx.x % per_group);
-    const int gcur = min(p.group, p.BH_kv - g0);
-    const int j = r_in / gcur;
-    bh = g0 + r_in % gcur;
+    int j;
+    grouped_unit(static_cast<int>(blockIdx.x), p.n_kv, p.BH_kv, p.group, j, bh);
     k0 = 128 * j;
     qi0 = causal ? max(0, k0 - p.off) / 64 : 0;  // first 64-row tile that sees this key tile
     n_qt = max(0, p.n_q - qi0);

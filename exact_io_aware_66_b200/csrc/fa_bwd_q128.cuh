@@ -125,12 +125,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
   // Scheduling as in fa_bwd_main: groups of p.group key/value heads sized for L2; inside a
   // group the key tiles with the most query tiles first (longest-processing-time order).
-  const int per_group = p.group * p.n_kv;
-  const int g0 = static_cast<int>(blockIdx.x / per_group) * p.group;
-  const int r_in = static_cast<int>(blockIdx.x % per_group);
-  const int gcur = min(p.group, p.BH_kv - g0);
-  const int j = r_in / gcur;
-  const int bh = g0 + r_in % gcur;  // key/value head
+  int j, bh;  // key tile, key/value head
+  grouped_unit(static_cast<int>(blockIdx.x), p.n_kv, p.BH_kv, p.group, j, bh);
   const int k0 = 128 * j;
   // First 128-row query tile with a query that sees a key of this tile (j <= i + off); the
   // iterations run over every query head sharing this key/value head, times its query tiles.

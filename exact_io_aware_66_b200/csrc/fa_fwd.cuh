@@ -96,19 +96,40 @@ struct FwdParams {
   unsigned long long limit_ns = FA_SPIN_LIMIT_NS;
 };
 
+// Work unit `b` of a grid covering n_heads heads x n_tiles tiles, heads taken in groups of
+// `group` (sized on the host so that a group's shared operands stay in L2 while its units run;
+// the hardware hands out blocks roughly in index order, so a group's units run together). Inside
+// a group, tile rank 0 (the heaviest tile) comes first for every head of the group, then rank 1,
+// and so on (longest-processing-time order). When `group` does not divide n_heads, the smaller
+// group goes first: run last, its heaviest units would start when every other unit has been
+// handed out and end well after them.
+__device__ __forceinline__ void grouped_unit(int b, int n_tiles, int n_heads, int group, int& rank,
+                                             int& head) {
+  const int rem = n_heads % group;
+  const int first = rem * n_tiles;  // units of the smaller group
+  int g0, gcur, r;
+  if (b < first) {
+    g0 = n_heads - rem;
+    gcur = rem;
+    r = b;
+  } else {
+    b -= first;
+    g0 = (b / (group * n_tiles)) * group;
+    gcur = group;
+    r = b % (group * n_tiles);
+  }
+  rank = r / gcur;
+  head = g0 + r % gcur;
+}
+
 // Work unit of CTA `cta` in a forward grid of n_qblocks * BH CTAs: query block qb of query head
-// bh. Heads are taken in groups of `hgroup` consecutive query heads, sized on the host so that a
-// group's K and V stay in L2 while its CTAs run; inside a group the heaviest query blocks
-// (causal work grows with the block index) come first, cycling over the group's heads
-// (longest-processing-time order).
+// bh, in groups of `hgroup` query heads whose K and V stay in L2; causal work grows with the
+// query block index, so the last blocks are the heaviest.
 __device__ __forceinline__ void fwd_work_unit(int cta, int n_qblocks, int BH, int hgroup, int& qb,
                                               int& bh) {
-  const int per_group = hgroup * n_qblocks;
-  const int g0 = (cta / per_group) * hgroup;
-  const int r = cta % per_group;
-  const int gcur = min(hgroup, BH - g0);
-  qb = n_qblocks - 1 - r / gcur;
-  bh = g0 + r % gcur;
+  int rank;
+  grouped_unit(cta, n_qblocks, BH, hgroup, rank, bh);
+  qb = n_qblocks - 1 - rank;
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
