@@ -120,38 +120,79 @@ REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_powe
 
 
 class ClockSampler:
+    """SM clocks and clock-event reasons during the timed region, read-only.
+
+    nvidia-smi samples every 200 ms; a short timed region can end before its first sample, so
+    an NVML polling thread (10 ms) runs beside it and its samples are reported when nvidia-smi
+    has none."""
+
+    NVML_BITS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+                 "sw_power_cap": 0x4}
+
     def __init__(self, device: int):
         self.proc = None
-        self.path = None
+        self.thread = None
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         except Exception:
             self.gpu = str(device)
 
+    def _nvml_loop(self):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(self.gpu)
+                maxmhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+                while not self.stop_evt.is_set():
+                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    bits = reasons_fn(h)
+                    self.nvml.append((time.time(), float(mhz), float(maxmhz), int(bits)))
+                    self.stop_evt.wait(0.01)
+            finally:
+                pynvml.nvmlShutdown()
+        except Exception:
+            pass
+
     def start(self):
+        import threading
+
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
              "clocks_event_reasons.sw_power_cap")
         try:
-            self.out = open(os.devnull, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200",
                  "-i", self.gpu], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+        self.nvml = []
+        self.stop_evt = threading.Event()
+        self.thread = threading.Thread(target=self._nvml_loop, daemon=True)
+        self.thread.start()
+        t0 = time.time()  # let the NVML thread take its first sample before the region starts
+        while not self.nvml and self.thread.is_alive() and time.time() - t0 < 2.0:
+            time.sleep(0.002)
+        self.t_region = time.time()
 
     def stop(self) -> dict | None:
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except Exception:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
+        out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
         mhz, maxmhz, reasons = [], [], set()
-        for line in out.strip().splitlines():
+        for line in (out or "").strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 8:
                 continue
@@ -163,10 +204,18 @@ class ClockSampler:
             for name, val in zip(REASONS, parts[4:8]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
+        source = "nvidia-smi"
+        if not mhz and self.thread is not None:
+            source = "nvml"
+            inside = [x for x in self.nvml if x[0] >= self.t_region] or self.nvml
+            for _, m, mx, bits in inside:
+                mhz.append(m)
+                maxmhz.append(mx)
+                reasons.update(n for n, b in self.NVML_BITS.items() if bits & b)
         if not mhz:
             return None
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxmhz),
-                "reasons": sorted(reasons), "samples": len(mhz)}
+                "reasons": sorted(reasons), "samples": len(mhz), "source": source}
 
 
 # --------------------------------------------------------------------------------------------
