@@ -118,6 +118,7 @@ struct DeviceState {
   std::atomic<bool> bwd_attr[2][2][2] = {};
   std::atomic<bool> bwd128_attr[4] = {};  // [2 (d = 128) + causal]
   std::atomic<bool> bwd256_attr[2] = {};  // [causal]
+  int n_sm = 0;  // multiprocessors (grid of the persistent kernels)
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -161,6 +162,7 @@ DeviceState* device_state(fa_status* st) {
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
     ds.is_sm100 = (major == 10 && minor == 0);
+    cudaDeviceGetAttribute(&ds.n_sm, cudaDevAttrMultiProcessorCount, dev);
     ds.checked = true;
   }
   if (!ds.is_sm100) {
@@ -379,10 +381,12 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
     const unsigned nb = static_cast<unsigned>(prep_blocks);
     if (s.d == 96)
       fa::fa_bwd_preprocess<96><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc, Dvec,
-                                                                     lse2, rows, N, n64);
+                                                                     lse2, rows, N, n64,
+        nullptr);
     else
       fa::fa_bwd_preprocess<D><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc, Dvec,
-                                                                    lse2, rows, N, n64);
+                                                                    lse2, rows, N, n64,
+        nullptr);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd preprocess launch");
@@ -459,6 +463,7 @@ fa_status launch_bwd_q128(DeviceState* ds, const void* q, const void* k, const v
   float* dq_acc = reinterpret_cast<float*>(ws);
   float* Dvec = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_D(BH, N, s.d));
   float* lse2 = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_lse2(BH, N, s.d));
+  int* sched = reinterpret_cast<int*>(ws + fa::bwd_ws_offset_sched(BH, N, s.d));
   const int n64 = static_cast<int>(fa::bwd_n64(N));
   const long long rows = 1LL * BH * N;
 
@@ -494,10 +499,12 @@ fa_status launch_bwd_q128(DeviceState* ds, const void* q, const void* k, const v
     const unsigned nb = static_cast<unsigned>(prep_blocks);
     if (s.d == 96)
       fa::fa_bwd_preprocess<96><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc, Dvec,
-                                                                     lse2, rows, N, n64);
+                                                                     lse2, rows, N, n64,
+        sched);
     else
       fa::fa_bwd_preprocess<D><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc,
-                                                                    Dvec, lse2, rows, N, n64);
+                                                                    Dvec, lse2, rows, N, n64,
+        sched);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd preprocess launch");
@@ -522,12 +529,17 @@ fa_status launch_bwd_q128(DeviceState* ds, const void* q, const void* k, const v
   p.scale = s.scale;
   p.scale_log2 = s.scale * 1.4426950408889634f;
   apply_stall(2, p);
-  const long long grid = 1LL * p.n_kv * BHkv;
-  if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  // persistent: one CTA per SM (at most one per unit), units handed out by the counter
+  const long long units = 1LL * p.n_kv * BHkv;
+  if (units >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  p.n_units = static_cast<int>(units);
+  p.sched_counter = sched;
+  const int n_sm = ds->n_sm > 0 ? ds->n_sm : 148;
+  const unsigned grid = static_cast<unsigned>(units < n_sm ? units : n_sm);
   {
     ProfileScope prof(2, stream);
-    kern<<<static_cast<unsigned>(grid), fa::kBwdThreads, L::kBytes, stream>>>(
-        tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv, p);
+    kern<<<grid, fa::kBwdThreads, L::kBytes, stream>>>(tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv,
+                                                        p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd main (q128) launch");
@@ -596,7 +608,8 @@ fa_status launch_bwd_d256(DeviceState* ds, const void* q, const void* k, const v
     ProfileScope prof(1, stream);
     fa::fa_bwd_preprocess<256><<<static_cast<unsigned>(prep_blocks), fa::kPrepThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dq_acc,
-        Dvec, lse2, rows, N, n64);
+        Dvec, lse2, rows, N, n64,
+        nullptr);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd preprocess launch");
@@ -952,6 +965,7 @@ struct NoAllocDevice {
   int* status = nullptr;    // device address of g_noalloc_status on this device
   bool bwd_attr[2][2][2] = {};
   bool bwd128_attr[4] = {};
+  int n_sm = 0;
   bool bwd256_attr[2] = {};
 };
 
@@ -1134,10 +1148,12 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
       if (e != cudaSuccess) return cuda_err(e, "cudaGetSymbolAddress(status)");
       nd.scratch = scratch;
       nd.status = static_cast<int*>(status);
+      cudaDeviceGetAttribute(&nd.n_sm, cudaDevAttrMultiProcessorCount, dev);
       nd.ready = true;
     }
     local.status = nd.status;
     local.checked = local.is_sm100 = true;
+    local.n_sm = nd.n_sm;
     copy_flags(local.bwd_attr, nd.bwd_attr);
     for (int c = 0; c < 4; ++c) local.bwd128_attr[c].store(nd.bwd128_attr[c]);
     for (int c = 0; c < 2; ++c) local.bwd256_attr[c].store(nd.bwd256_attr[c]);

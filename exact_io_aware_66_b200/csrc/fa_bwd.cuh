@@ -33,10 +33,11 @@
 
 namespace fa {
 
-// Workspace layout (all fp32, each section 256-byte aligned):
-//   dQ_acc [BH, N, d] | D [BH, N64] | lse2 [BH, N64]
+// Workspace layout (each section 256-byte aligned):
+//   dQ_acc [BH, N, d] fp32 | D [BH, N64] fp32 | lse2 [BH, N64] fp32 | unit counter (int)
 // where N64 = N rounded up to a multiple of 64, so every row of D and lse2 starts on a
-// 256-byte boundary (TMA needs 16-byte aligned row strides).
+// 256-byte boundary (TMA needs 16-byte aligned row strides). The counter hands out work units
+// to the persistent 128-row backward kernel; the preprocess kernel zeroes it.
 __host__ __device__ inline size_t bwd_align256(size_t x) { return (x + 255) / 256 * 256; }
 inline size_t bwd_n64(int N) { return (static_cast<size_t>(N) + 63) / 64 * 64; }
 inline size_t bwd_ws_offset_D(size_t BH, int N, int d) {
@@ -45,8 +46,11 @@ inline size_t bwd_ws_offset_D(size_t BH, int N, int d) {
 inline size_t bwd_ws_offset_lse2(size_t BH, int N, int d) {
   return bwd_ws_offset_D(BH, N, d) + bwd_align256(BH * bwd_n64(N) * 4);
 }
-inline size_t bwd_workspace_bytes(size_t BH, int N, int d) {
+inline size_t bwd_ws_offset_sched(size_t BH, int N, int d) {
   return bwd_ws_offset_lse2(BH, N, d) + bwd_align256(BH * bwd_n64(N) * 4);
+}
+inline size_t bwd_workspace_bytes(size_t BH, int N, int d) {
+  return bwd_ws_offset_sched(BH, N, d) + 256;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -60,12 +64,13 @@ __global__ void __launch_bounds__(kPrepThreads)
     fa_bwd_preprocess(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                       const float* __restrict__ lse, float* __restrict__ dq_acc,
                       float* __restrict__ Dvec, float* __restrict__ lse2, long long rows, int N,
-                      int n64) {
+                      int n64, int* __restrict__ counter) {
   constexpr int TPR = D <= 64 ? 8 : (D <= 128 ? 16 : 32);  // threads per row
   static_assert(D % 8 == 0 && D / 8 <= TPR, "preprocess row split");
   const long long t = static_cast<long long>(blockIdx.x) * kPrepThreads + threadIdx.x;
   const long long row = t / TPR;
   const int part = static_cast<int>(t % TPR);
+  if (t == 0 && counter != nullptr) *counter = 0;  // unit counter of the persistent main kernel
   float acc = 0.f;
   if (row < rows && part * 8 < D) {
     const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
@@ -174,6 +179,10 @@ struct BwdParams {
   // the kernel unwinds with FA_ERR_TIMEOUT. limit_ns bounds the MMA warp's waits.
   int dbg_skip = -1;
   unsigned long long limit_ns = FA_SPIN_LIMIT_NS;
+  // Persistent kernels (fa_bwd_q128.cuh): units n_kv * BH_kv in all, the first gridDim.x taken
+  // by block index, the rest handed out by this zeroed counter.
+  int n_units = 0;
+  int* sched_counter = nullptr;
 };
 
 template <int D, bool CAUSAL, bool DROPOUT>
