@@ -359,4 +359,37 @@ __host__ __device__ constexpr uint32_t sw128_offset(uint32_t row, uint32_t chunk
   return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
+// ------------------------------------------------------------------------------------------
+// Cluster launch control (sm_100): a running CTA asks the hardware to cancel a CTA of its own
+// grid that has not been launched yet, and then does that CTA's work itself. Launched with one
+// CTA per work unit, a kernel whose CTAs keep asking runs persistently, and the units still go
+// out in launch order, one at a time, to whichever SM frees up first. One request at a time per
+// CTA; after a request that cancelled nothing the CTA must not ask again.
+// ------------------------------------------------------------------------------------------
+// Issues a request; the 16-byte response lands at `resp` (16-byte aligned shared memory) and
+// completes 16 bytes of transaction count on `bar` (arm it with mbar_arrive_expect_tx first).
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 "
+      "[%0], [%1];" ::"r"(resp),
+      "r"(bar)
+      : "memory");
+}
+// Reads a completed response: blockIdx.x of the cancelled CTA, or -1 when none was cancelled.
+// The response buffer may be reused by the next request afterwards.
+__device__ __forceinline__ int clc_cancelled_x(uint32_t resp) {
+  uint32_t x = 0, y = 0, z = 0, ok = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 c;\n\t"
+      "ld.shared.b128 c, [%4];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, c;\n\t"
+      "selp.u32 %3, 1, 0, p;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid.v4.b32.b128 {%0, %1, %2, _}, c;\n\t}"
+      : "+r"(x), "+r"(y), "+r"(z), "=r"(ok)
+      : "r"(resp)
+      : "memory");
+  fence_proxy_async_smem();
+  return ok ? static_cast<int>(x) : -1;
+}
+
 }  // namespace fa
