@@ -100,7 +100,8 @@ typedef struct {
 fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
                     const fa_attn_shape* shape, const fa_dropout* dropout, void* stream);
 
-/* Workspace bytes fa_bwd_ex needs (fp32 dQ accumulator and row terms for B*H*N_q rows); 0 for an
+/* Workspace bytes fa_bwd_ex needs (fp32 dQ accumulator and row terms for B*H*N_q rows, and the
+ * work-unit counter of the persistent backward kernel); 0 for an
  * invalid shape. */
 size_t fa_bwd_ex_workspace_size(const fa_attn_shape* shape);
 
@@ -117,13 +118,16 @@ fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int N, int d, float scale, int causal, void* stream);
 
-/* Bytes of device workspace fa_bwd needs for these sizes (fp32 dQ accumulator [B,H,N,d] and
- * the fp32 row term D [B,H,N]). Returns 0 for invalid sizes. */
+/* Bytes of device workspace fa_bwd needs for these sizes (fp32 dQ accumulator [B,H,N,d], the
+ * fp32 row terms D and -lse*log2(e) [B,H,N], and a counter that hands out work units to the
+ * persistent backward kernel; the first kernel of each call zeroes it). Returns 0 for invalid
+ * sizes. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
 /* Backward. Inputs q, k, v, o (from fa_fwd), dO and lse (from fa_fwd); outputs dq, dk, dv
  * (bf16 [B,H,N,d]). workspace: caller-owned device memory of at least
- * fa_bwd_workspace_size(B,H,N,d) bytes, 16-byte aligned; its contents on entry do not matter. */
+ * fa_bwd_workspace_size(B,H,N,d) bytes, 16-byte aligned; its contents on entry do not matter.
+ * Calls that share a workspace must be ordered (one stream, or events between streams). */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                  const float* lse, void* dq, void* dk, void* dv, void* workspace,
                  size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
@@ -134,7 +138,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * reserved the GPU's memory for its own pool and hands out no workspace, or a service that
  * must not allocate after start-up to keep its latency and memory footprint fixed. They call
  * this instead of fa_bwd: same arguments without the workspace, same results.
- * The scratch (fp32 dQ accumulator, per-row terms) is a 64 MiB array built into the library:
+ * The scratch (fp32 dQ accumulator, per-row terms, work-unit counter) is a 64 MiB array built
+ * into the library:
  * every GPU that loads the library holds it until the process exits. Sizes whose
  * fa_bwd_workspace_size exceeds 64 MiB (67108864 bytes) are rejected with FA_ERR_UNSUPPORTED
  * and nothing is launched. This call performs no cudaMalloc, cudaFree or other allocation.
