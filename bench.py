@@ -518,7 +518,6 @@ def main():
     fa.fa_check_status(stream)
     cfg = workload_config(w, world, args.dropout, args.fp8)
     flops_step = cfg["flops_per_step"]
-    launches_per_step = (2 if args.fp8 else 1) + (3 if backward else 0)
 
     # ---- timed region: K steps, L2 flushed before each (outside the event pairs) ----
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -680,7 +679,7 @@ def main():
             "per_config": per_config,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": sum(v["launches"] for v in kern.values()),
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
