@@ -13,8 +13,10 @@
 // the TMA loads). The PV product wants V with the key index contiguous (K-major B operand), so
 // V is first transposed into a workspace [B*H_kv][d][N_kv padded to 16] by fa_fp8_transpose_v.
 //
-// Roles (16 warps), TMEM and the issue order are those of fa_fwd.cuh; P takes 32 TMEM columns
-// (four E4M3 per column) at the start of its S buffer.
+// Roles (16 warps), TMEM, the issue order and the persistent scheduling (cluster launch control,
+// units handed to the roles through a two-slot ring, barrier phases counted over the CTA's
+// run) are those of fa_fwd.cuh; P takes 32 TMEM columns (four E4M3 per column) at the start of
+// its S buffer.
 #pragma once
 #include <cuda_fp8.h>
 
@@ -32,20 +34,30 @@ struct Fp8Layout {
   static constexpr int kKV = 2 * kTile;
   static constexpr int kO = kKV + kStages * kTile;  // O0, O1 staging
   static constexpr int kBars = kO + 2 * kOTile;
-  static constexpr int kNumBars = 1 + 2 * kStages + 11;
+  static constexpr int kNumBars = 1 + 2 * kStages + 19;
   static constexpr int kRowL = kBars + kNumBars * 8;
-  static constexpr int kTmemSlot = kRowL + 2 * 128 * 4;
+  static constexpr int kSched = kRowL + 2 * 128 * 4;       // two unit indices
+  static constexpr int kClc = (kSched + 8 + 15) / 16 * 16;  // 16-byte launch-control reply
+  static constexpr int kTmemSlot = kClc + 16;
   static constexpr int kBytes = kTmemSlot + 16;
   static constexpr int kAlloc = kBytes + 1024;
 
+  // barriers as in FwdLayout
   static constexpr int bQ = 0;
   static constexpr int bKvFull = 1;
   static constexpr int bKvEmpty = 1 + kStages;
   static constexpr int bSFull = 1 + 2 * kStages;
   static constexpr int bPFull = bSFull + 2;
-  static constexpr int bODone = bSFull + 6;
-  static constexpr int bFinal = bSFull + 8;
-  static constexpr int bDrain = bSFull + 10;
+  static constexpr int bODone = bSFull + 4;
+  static constexpr int bFinal = bSFull + 6;
+  static constexpr int bOFree = bSFull + 8;
+  static constexpr int bRowFree = bSFull + 10;
+  static constexpr int bSchedFull = bSFull + 12;
+  static constexpr int bSchedEmpty = bSFull + 14;
+  static constexpr int bQEmpty = bSFull + 16;
+  static constexpr int bClc = bSFull + 17;
+  static constexpr int bDrain = bSFull + 18;
+  static constexpr int kSchedReaders = 13;
 };
 static_assert(Fp8Layout::kAlloc <= 227 * 1024, "fp8 forward shared memory");
 
@@ -117,20 +129,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint8_t* gbase = smem_raw + (sbase - raw);
   auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * i; };
   float* s_rowl = reinterpret_cast<float*>(gbase + L::kRowL);
+  volatile int* sched = reinterpret_cast<volatile int*>(gbase + L::kSched);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  int qb, bh;
-  fwd_work_unit(static_cast<int>(blockIdx.x), p.n_qblocks, p.BH, p.hgroup, qb, bh);
-  const int bh_kv = bh / p.group;
-  const int q0 = qb * 256;
   const int nkv = (p.N_kv + 127) / 128;
-  int n_t[2];
+  struct Unit {  // as in fa_fwd_kernel
+    int q0, bh, n_t[2];
+  };
+  auto unit_of = [&](int u) {
+    Unit w;
+    int qb;
+    fwd_work_unit(u, p.n_qblocks, p.BH, p.hgroup, qb, w.bh);
+    w.q0 = qb * 256;
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int last_key = q0 + 128 * t + 127 + p.off;
-    n_t[t] = !CAUSAL ? nkv : (last_key < 0 ? 0 : min(nkv, last_key / 128 + 1));
-  }
+    for (int t = 0; t < 2; ++t) {
+      const int last_key = w.q0 + 128 * t + 127 + p.off;
+      w.n_t[t] = !CAUSAL ? nkv : (last_key < 0 ? 0 : min(nkv, last_key / 128 + 1));
+    }
+    return w;
+  };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -144,7 +162,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(bar(L::bPFull + t), 128);
       mbar_init(bar(L::bODone + t), 1);
       mbar_init(bar(L::bFinal + t), 128);
+      mbar_init(bar(L::bOFree + t), 128);
+      mbar_init(bar(L::bRowFree + t), 128);
+      mbar_init(bar(L::bSchedFull + t), 1);
+      mbar_init(bar(L::bSchedEmpty + t), L::kSchedReaders);
     }
+    mbar_init(bar(L::bQEmpty), 1);
+    mbar_init(bar(L::bClc), 1);
     mbar_init(bar(L::bDrain), 1);
     fence_barrier_init();
   }
@@ -163,165 +187,204 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::kTmemSlot);
 
+  constexpr int kGaveUp = -2;
+  auto warp_next_unit = [&](int s) -> int {
+    if (!warp_wait(bar(L::bSchedFull + (s & 1)), (s >> 1) & 1, abort_flag)) return kGaveUp;
+    const int u = sched[s & 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::bSchedEmpty + (s & 1)));
+    return u;
+  };
+
   if (warp < 8) {
     // ------------------------------------------------------------------ softmax ----------
     setmaxnreg_inc<R::kSoftmax>();
     const int t = warp >> 2;
     const int row = threadIdx.x & 127;
     const uint32_t tS = tmem + t * 128 + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const int q_row = q0 + t * 128 + row;
     const float sl2 = p.scale_log2;
-    float m = -INFINITY;
-    float l = 0.f;   // sum of the fp32 exponentials: gives lse
-    float lr = 0.f;  // sum of the same exponentials rounded to E4M3: normalises O
-    for (int j = 0; j < n_t[t]; ++j) {
-      if (!warp_wait(bar(L::bSFull + t), j & 1, abort_flag)) {
-        fail(p.status, abort_flag, 5);
+    int sc = 0;  // S tiles of this query tile in earlier units
+    bool ok = true;
+    for (int si = 0, uc = 0; ok; ++si, ++uc) {
+      const int u = warp_next_unit(si);
+      if (u == kGaveUp) { ok = false; break; }
+      if (u < 0) break;
+      const Unit U = unit_of(u);
+      const int q0 = U.q0, bh = U.bh, n = U.n_t[t];
+      const int q_row = q0 + t * 128 + row;
+      float m = -INFINITY;
+      float l = 0.f;   // sum of the fp32 exponentials: gives lse
+      float lr = 0.f;  // sum of the same exponentials rounded to E4M3: normalises O
+      for (int j = 0; j < n; ++j) {
+        if (!warp_wait(bar(L::bSFull + t), (sc + j) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t s[128];
+        tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+        tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+        tmem_ld_wait();
+        reg_fence(s);
+        const int kv0 = j * 128;
+        const bool need_mask = (CAUSAL && kv0 + 127 > q0 + t * 128 + p.off) || (kv0 + 128 > p.N_kv);
+        if (need_mask) {
+          const int lim = CAUSAL ? min(q_row + 1 + p.off, p.N_kv) : p.N_kv;
+  #pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
+        }
+        float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
+        float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
+  #pragma unroll
+        for (int c = 4; c < 128; c += 8) {
+          mx0 = max3f(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+          mx1 = max3f(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+          mx2 = max3f(mx2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+          mx3 = max3f(mx3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+        }
+        // Threshold update of the running max as in fa_fwd.cuh: weights stay below 2^8, inside
+        // E4M3's range (448).
+        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        float alpha = 1.0f;
+        if ((m_tile - m) * sl2 > kRescaleLog2) {
+          alpha = ex2_approx((m - m_tile) * sl2);
+          m = m_tile;
+        }
+        const float nb = m == -INFINITY ? 0.f : -m * sl2;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), nbx2 = f2_pack(nb, nb);
+        uint64_t lsum[2] = {0, 0}, rsum[2] = {0, 0};
+        uint32_t pk[32];
+  #pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          float a0, a1, a2, a3;
+          f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, nbx2), a0, a1);
+          f2_unpack(f2_fma(f2_pack_u(s[c + 2], s[c + 3]), sl2x2, nbx2), a2, a3);
+          const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
+          const float e2 = ex2_approx(a2), e3 = ex2_approx(a3);
+          float r0, r1, r2, r3;
+          const uint32_t lo = e4m3x2_round(e0, e1, r0, r1);
+          const uint32_t hi = e4m3x2_round(e2, e3, r2, r3);
+          pk[c / 4] = lo | (hi << 16);
+          const int acc = (c >> 2) & 1;
+          lsum[acc] = f2_add(lsum[acc], f2_add(f2_pack(e0, e1), f2_pack(e2, e3)));
+          rsum[acc] = f2_add(rsum[acc], f2_add(f2_pack(r0, r1), f2_pack(r2, r3)));
+        }
+        {
+          const uint64_t ls = f2_add(lsum[0], lsum[1]);
+          const uint64_t rs = f2_add(rsum[0], rsum[1]);
+          float x0, x1, y0, y1;
+          f2_unpack(ls, x0, x1);
+          f2_unpack(rs, y0, y1);
+          l = l * alpha + (x0 + x1);
+          lr = lr * alpha + (y0 + y1);
+        }
+        tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+        // O correction (PV(j-1) has completed: S(j) was issued after it).
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+          const uint32_t tO = tmem + 256 + t * 128 + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+  #pragma unroll
+          for (int c = 0; c < 128; c += 32) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(tO + c, o);
+            tmem_ld_wait();
+            reg_fence(o);
+            const uint64_t a2 = f2_pack(alpha, alpha);
+  #pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const uint64_t r = f2_mul(f2_pack_u(o[i], o[i + 1]), a2);
+              o[i] = static_cast<uint32_t>(r);
+              o[i + 1] = static_cast<uint32_t>(r >> 32);
+            }
+            tmem_st_32x32b_x32(tO + c, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::bPFull + t));
+      }
+      if (!ok) break;
+      sc += n;
+      // row sums for the epilogue, once it has read the previous unit's
+      if (uc > 0 && !warp_wait(bar(L::bRowFree + t), (uc - 1) & 1, abort_flag)) {
+        ok = false;
         break;
       }
-      tc_fence_after();
-      uint32_t s[128];
-      tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-      tmem_ld_wait();
-      reg_fence(s);
-      const int kv0 = j * 128;
-      const bool need_mask = (CAUSAL && kv0 + 127 > q0 + t * 128 + p.off) || (kv0 + 128 > p.N_kv);
-      if (need_mask) {
-        const int lim = CAUSAL ? min(q_row + 1 + p.off, p.N_kv) : p.N_kv;
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
-      }
-      float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
-      float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
-#pragma unroll
-      for (int c = 4; c < 128; c += 8) {
-        mx0 = max3f(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-        mx1 = max3f(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
-        mx2 = max3f(mx2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
-        mx3 = max3f(mx3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
-      }
-      // Threshold update of the running max as in fa_fwd.cuh: weights stay below 2^8, inside
-      // E4M3's range (448).
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-      float alpha = 1.0f;
-      if ((m_tile - m) * sl2 > kRescaleLog2) {
-        alpha = ex2_approx((m - m_tile) * sl2);
-        m = m_tile;
-      }
-      const float nb = m == -INFINITY ? 0.f : -m * sl2;
-      const uint64_t sl2x2 = f2_pack(sl2, sl2), nbx2 = f2_pack(nb, nb);
-      uint64_t lsum[2] = {0, 0}, rsum[2] = {0, 0};
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        float a0, a1, a2, a3;
-        f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, nbx2), a0, a1);
-        f2_unpack(f2_fma(f2_pack_u(s[c + 2], s[c + 3]), sl2x2, nbx2), a2, a3);
-        const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
-        const float e2 = ex2_approx(a2), e3 = ex2_approx(a3);
-        float r0, r1, r2, r3;
-        const uint32_t lo = e4m3x2_round(e0, e1, r0, r1);
-        const uint32_t hi = e4m3x2_round(e2, e3, r2, r3);
-        pk[c / 4] = lo | (hi << 16);
-        const int acc = (c >> 2) & 1;
-        lsum[acc] = f2_add(lsum[acc], f2_add(f2_pack(e0, e1), f2_pack(e2, e3)));
-        rsum[acc] = f2_add(rsum[acc], f2_add(f2_pack(r0, r1), f2_pack(r2, r3)));
-      }
-      {
-        const uint64_t ls = f2_add(lsum[0], lsum[1]);
-        const uint64_t rs = f2_add(rsum[0], rsum[1]);
-        float x0, x1, y0, y1;
-        f2_unpack(ls, x0, x1);
-        f2_unpack(rs, y0, y1);
-        l = l * alpha + (x0 + x1);
-        lr = lr * alpha + (y0 + y1);
-      }
-      tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-      // O correction (PV(j-1) has completed: S(j) was issued after it).
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        const uint32_t tO = tmem + 256 + t * 128 + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-#pragma unroll
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(tO + c, o);
-          tmem_ld_wait();
-          reg_fence(o);
-          const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const uint64_t r = f2_mul(f2_pack_u(o[i], o[i + 1]), a2);
-            o[i] = static_cast<uint32_t>(r);
-            o[i + 1] = static_cast<uint32_t>(r >> 32);
-          }
-          tmem_st_32x32b_x32(tO + c, o);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(L::bPFull + t));
+      s_rowl[t * 128 + row] = lr;
+      mbar_arrive(bar(L::bFinal + t));
+      if (!*abort_flag && q_row < p.N)
+        p.lse[static_cast<size_t>(bh) * p.N + q_row] =
+            l > 0.f ? (m * sl2 + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
     }
-    s_rowl[t * 128 + row] = lr;
-    mbar_arrive(bar(L::bFinal + t));
-    if (!*abort_flag && q_row < p.N)
-      p.lse[static_cast<size_t>(bh) * p.N + q_row] =
-          l > 0.f ? (m * sl2 + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
+    if (!ok) fail(p.status, abort_flag, 5);
   } else if (warp < 12) {
     // ----------------------------------------------------------------- epilogue ----------
     setmaxnreg_dec<R::kEpilogue>();
     const int row = threadIdx.x - 256;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int oc[2] = {0, 0};  // PV products of each tile in earlier units (phases of bODone)
     bool ok = true;
-    for (int t = 0; t < 2 && ok; ++t) {
-      // O has its own staging area, so an empty tile needs no ordering against the Q load.
-      if (!warp_wait(bar(L::bFinal + t), 0, abort_flag) ||
-          (n_t[t] > 0 && !warp_wait(bar(L::bODone + t), (n_t[t] - 1) & 1, abort_flag))) {
-        fail(p.status, abort_flag, 5);
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const float lr_row = s_rowl[t * 128 + row];
-      const float inv_l = lr_row > 0.f ? p.o_scale / lr_row : 0.f;
-      const bool empty_tile = n_t[t] == 0;
-      const uint32_t tO = tmem + 256 + t * 128 + lane_off;
-      uint8_t* stage = gbase + L::kO + t * L::kOTile;
-#pragma unroll
-      for (int c = 0; c < 128; c += 32) {
-        uint32_t o[32];
-        if (!empty_tile) {
-          tmem_ld_32x32b_x32(tO + c, o);
-          tmem_ld_wait();
-          reg_fence(o);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
+    for (int si = 0, uc = 0; ok; ++si, ++uc) {
+      const int u = warp_next_unit(si);
+      if (u == kGaveUp) { ok = false; break; }
+      if (u < 0) break;
+      const Unit U = unit_of(u);
+      for (int t = 0; t < 2; ++t) {
+        const int n = U.n_t[t];
+        if (!warp_wait(bar(L::bFinal + t), uc & 1, abort_flag) ||
+            (n > 0 && !warp_wait(bar(L::bODone + t), (oc[t] + n - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
         }
+        oc[t] += n;
+        tc_fence_after();
+        const float lr_row = s_rowl[t * 128 + row];
+        mbar_arrive(bar(L::bRowFree + t));
+        const float inv_l = lr_row > 0.f ? p.o_scale / lr_row : 0.f;
+        const uint32_t tO = tmem + 256 + t * 128 + lane_off;
+        uint8_t* stage = gbase + L::kO + t * L::kOTile;
+        if (lane == 0) bulk_wait_group_read0();  // the previous unit's store has read it
+        __syncwarp();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
-          v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
-          v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
-          v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
-          const int chunk = c / 8 + q;  // 0 .. 15
-          *reinterpret_cast<uint4*>(stage + (chunk >> 3) * L::kOBoxBytes +
-                                    sw128_offset(row, chunk & 7)) = v;
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t o[32];
+          if (n > 0) {
+            tmem_ld_32x32b_x32(tO + c, o);
+            tmem_ld_wait();
+            reg_fence(o);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0u;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+            const int chunk = c / 8 + q;  // 0 .. 15
+            *reinterpret_cast<uint4*>(stage + (chunk >> 3) * L::kOBoxBytes +
+                                      sw128_offset(row, chunk & 7)) = v;
+          }
         }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        for (int b = 0; b < p.o_boxes; ++b)
-          tma_store_3d(&tmO, sbase + L::kO + t * L::kOTile + b * L::kOBoxBytes + (warp & 3) * 4096,
-                       64 * b, q0 + t * 128 + (warp & 3) * 32, bh);
-        bulk_commit_group();
+        tc_fence_before();
+        mbar_arrive(bar(L::bOFree + t));  // O(t) is out of TMEM: the next unit may overwrite it
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int b = 0; b < p.o_boxes; ++b)
+            tma_store_3d(&tmO,
+                         sbase + L::kO + t * L::kOTile + b * L::kOBoxBytes + (warp & 3) * 4096,
+                         64 * b, U.q0 + t * 128 + (warp & 3) * 32, U.bh);
+          bulk_commit_group();
+        }
       }
     }
-    if (lane == 0) bulk_wait_group_read0();
+    if (!ok) fail(p.status, abort_flag, 5);
+    if (lane == 0) bulk_wait_group0();
   } else {
     setmaxnreg_dec<R::kMma>();
     if (warp == 12 && lane == 0) {
@@ -329,12 +392,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       constexpr uint32_t idesc = idesc_e4m3_f32(128, 128);  // QK^T and PV: M = N = 128
       const uint64_t desc_q0 = sdesc_sw128(sbase + L::kQ, 16, 1024);
       const uint64_t desc_kv0 = sdesc_sw128(sbase + L::kKV, 16, 1024);
+      // tt: the CTA's K/V load number (K of key tile j is load tb + 2j, V^T load tb + 2j + 1)
       auto wait_full = [&](int tt) -> bool {
         return mbar_wait(bar(L::bKvFull + tt % ST), (tt / ST) & 1, abort_flag);
       };
-      auto issue_s = [&](int t, int j) {
+      auto issue_s = [&](int t, int tt) {
         const uint64_t a0 = sdesc_advance(desc_q0, t * L::kTile);
-        const uint64_t b0 = sdesc_advance(desc_kv0, ((2 * j) % ST) * L::kTile);
+        const uint64_t b0 = sdesc_advance(desc_kv0, (tt % ST) * L::kTile);
         const uint32_t d = tmem + t * 128;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 32 E4M3 (32 bytes) of the head dimension per step
@@ -342,89 +406,138 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                      kk > 0 ? 1u : 0u);
         umma_commit(bar(L::bSFull + t));
       };
-      auto issue_pv = [&](int t, int j) {
-        const uint64_t b0 = sdesc_advance(desc_kv0, ((2 * j + 1) % ST) * L::kTile);
+      auto issue_pv = [&](int t, int tt, bool acc) {
+        const uint64_t b0 = sdesc_advance(desc_kv0, (tt % ST) * L::kTile);
         const uint32_t d = tmem + 256 + t * 128, a = tmem + t * 128;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 32 keys per step: 8 TMEM columns of P
-          umma_ts_f8(d, a + kk * 8, sdesc_advance(b0, kk * 32), idesc, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts_f8(d, a + kk * 8, sdesc_advance(b0, kk * 32), idesc, (acc || kk > 0) ? 1u : 0u);
         umma_commit(bar(L::bODone + t));
       };
-      bool ok = n_t[1] == 0 || (mbar_wait(bar(L::bQ), 0, abort_flag) && wait_full(0));
-      if (ok && n_t[1] > 0) {
+      bool ok = true;
+      int tb = 0;
+      int pc[2] = {0, 0};
+      for (int si = 0, uc = 0; ok; ++si, ++uc) {
+        if (!(ok = mbar_wait(bar(L::bSchedFull + (si & 1)), (si >> 1) & 1, abort_flag))) break;
+        const int u = sched[si & 1];
+        mbar_arrive(bar(L::bSchedEmpty + (si & 1)));
+        if (u < 0) break;
+        const Unit U = unit_of(u);
+        const int n0 = U.n_t[0], n1 = U.n_t[1];
+        if (!(ok = mbar_wait(bar(L::bQ), uc & 1, abort_flag) && (n1 == 0 || wait_full(tb)))) break;
         tc_fence_after();
-        if (n_t[0] > 0) issue_s(0, 0);
-        issue_s(1, 0);
-        umma_commit(bar(L::bKvEmpty + 0 % ST));
-      }
-      for (int j = 0; j < n_t[1] && ok; ++j) {
-        const int tv = 2 * j + 1, tk = 2 * j + 2;
-        if (!wait_full(tv)) { ok = false; break; }
-        tc_fence_after();
-        if (j < n_t[0]) {
-          if (!mbar_wait(bar(L::bPFull + 0), j & 1, abort_flag)) { ok = false; break; }
+        if (n1 > 0) {
+          if (n0 > 0) issue_s(0, tb);
+          issue_s(1, tb);
+          umma_commit(bar(L::bKvEmpty + tb % ST));
+        }
+        if (n1 <= 1) umma_commit(bar(L::bQEmpty));  // no further S reads this unit's Q
+        for (int j = 0; j < n1 && ok; ++j) {
+          const int tv = tb + 2 * j + 1, tk = tb + 2 * j + 2;
+          if (!wait_full(tv)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(0, j);
-        }
-        const bool more = j + 1 < n_t[1];
-        if (more) {
-          if (!wait_full(tk)) { ok = false; break; }
-          tc_fence_after();
-          if (j + 1 < n_t[0]) issue_s(0, j + 1);
-        }
-        if (!mbar_wait(bar(L::bPFull + 1), j & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(1, j);
-        umma_commit(bar(L::bKvEmpty + tv % ST));
-        if (more) {
-          issue_s(1, j + 1);
-          umma_commit(bar(L::bKvEmpty + tk % ST));
-        }
-      }
-      if (!ok) {
-        fail(p.status, abort_flag, 5);
-        volatile int never = 0;
-        umma_commit(bar(L::bDrain));
-        mbar_wait(bar(L::bDrain), 0, &never);
-      }
-    } else if (warp == 13 && lane == 0) {
-      // ------------------------------------------------------------------ TMA -------------
-      // The Q load is waited for by the MMA warp, or (when no key tile is visited) below.
-      mbar_arrive_expect_tx(bar(L::bQ), 2 * L::kTile);
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-        tma_load_3d(sbase + L::kQ + t * L::kTile, &tmQ, bar(L::bQ), 0, q0 + 128 * t, bh);
-      int issued = 0;
-      for (int j = 0; j < n_t[1]; ++j) {
-        bool ok = true;
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          const int tt = 2 * j + w;
-          const int st = tt % ST;
-          if (!mbar_wait(bar(L::bKvEmpty + st), ((tt / ST) & 1) ^ 1, abort_flag)) {
+          if (j < n0) {
+            if (!mbar_wait(bar(L::bPFull + 0), (pc[0] + j) & 1, abort_flag) ||
+                (j == 0 && uc > 0 && !mbar_wait(bar(L::bOFree + 0), (uc - 1) & 1, abort_flag))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(0, tv, j > 0);
+          }
+          const bool more = j + 1 < n1;
+          if (more) {
+            if (!wait_full(tk)) { ok = false; break; }
+            tc_fence_after();
+            if (j + 1 < n0) issue_s(0, tk);
+          }
+          if (!mbar_wait(bar(L::bPFull + 1), (pc[1] + j) & 1, abort_flag) ||
+              (j == 0 && uc > 0 && !mbar_wait(bar(L::bOFree + 1), (uc - 1) & 1, abort_flag))) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(L::bKvFull + st), L::kTile);
-          const uint32_t dst = sbase + L::kKV + st * L::kTile;
-          if (w == 0)
-            tma_load_3d(dst, &tmK, bar(L::bKvFull + st), 0, 128 * j, bh_kv);  // K rows
-          else
-            tma_load_3d(dst, &tmVt, bar(L::bKvFull + st), 128 * j, 0, bh_kv);  // V^T rows
-          issued = tt + 1;
+          tc_fence_after();
+          issue_pv(1, tv, j > 0);
+          umma_commit(bar(L::bKvEmpty + tv % ST));
+          if (more) {
+            issue_s(1, tk);
+            umma_commit(bar(L::bKvEmpty + tk % ST));
+            if (j + 2 == n1) umma_commit(bar(L::bQEmpty));
+          }
         }
-        if (!ok) {
-          fail(p.status, abort_flag, 5);
+        tb += 2 * n1;
+        pc[0] += n0;
+        pc[1] += n1;
+      }
+      if (!ok) fail(p.status, abort_flag, 5);
+      // every MMA issued completes before TMEM is freed (bounded wait)
+      volatile int never = 0;
+      umma_commit(bar(L::bDrain));
+      mbar_wait(bar(L::bDrain), 0, &never);
+    } else if (warp == 13 && lane == 0) {
+      // ------------------------------------------------- TMA, and the unit scheduler -------
+      bool ok = true;
+      int issued = 0, q_loads = 0, clc_n = 0;
+      bool clc_pending = false;
+      int u = static_cast<int>(blockIdx.x);
+      for (int si = 0; ok; ++si) {
+        if (!mbar_wait(bar(L::bSchedEmpty + (si & 1)), ((si >> 1) & 1) ^ 1, abort_flag)) {
+          ok = false;
           break;
         }
+        sched[si & 1] = u;
+        mbar_arrive(bar(L::bSchedFull + (si & 1)));
+        if (u < 0) break;
+        const Unit U = unit_of(u);
+        const int bh_kv = U.bh / p.group;
+        if (si > 0 && !mbar_wait(bar(L::bQEmpty), (si - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(L::bQ), 2 * L::kTile);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          tma_load_3d(sbase + L::kQ + t * L::kTile, &tmQ, bar(L::bQ), 0, U.q0 + 128 * t, U.bh);
+        q_loads = si + 1;
+        for (int j = 0; j < U.n_t[1] && ok; ++j) {
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const int tt = issued;
+            const int st = tt % ST;
+            if (!mbar_wait(bar(L::bKvEmpty + st), ((tt / ST) & 1) ^ 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(L::bKvFull + st), L::kTile);
+            const uint32_t dst = sbase + L::kKV + st * L::kTile;
+            if (w == 0)
+              tma_load_3d(dst, &tmK, bar(L::bKvFull + st), 0, 128 * j, bh_kv);  // K rows
+            else
+              tma_load_3d(dst, &tmVt, bar(L::bKvFull + st), 128 * j, 0, bh_kv);  // V^T rows
+            issued = tt + 1;
+          }
+        }
+        if (!ok) break;
+        // claim the next unit once this one's loads are all issued
+        mbar_arrive_expect_tx(bar(L::bClc), 16);
+        clc_try_cancel(sbase + L::kClc, bar(L::bClc));
+        clc_pending = true;
+        ++clc_n;
+        if (!mbar_wait(bar(L::bClc), (clc_n - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        clc_pending = false;
+        u = clc_cancelled_x(sbase + L::kClc);
       }
-      if (*abort_flag || n_t[1] == 0) {
-        // Let the loads in flight land before shared memory is released.
-        volatile int never = 0;
-        for (int tt = max(0, issued - ST); tt < issued; ++tt)
-          mbar_wait(bar(L::bKvFull + tt % ST), (tt / ST) & 1, &never);
-        mbar_wait(bar(L::bQ), 0, &never);
-      }
+      if (!ok) fail(p.status, abort_flag, 5);
+      // loads in flight and a pending launch-control reply land before the CTA exits
+      volatile int never = 0;
+#pragma unroll 1
+      for (int tt = max(0, issued - ST); tt < issued; ++tt)
+        mbar_wait(bar(L::bKvFull + tt % ST), (tt / ST) & 1, &never);
+      if (q_loads > 0) mbar_wait(bar(L::bQ), (q_loads - 1) & 1, &never);
+      if (clc_pending) mbar_wait(bar(L::bClc), (clc_n - 1) & 1, &never);
     }
   }
   tc_fence_before();
