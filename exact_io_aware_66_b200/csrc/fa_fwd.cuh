@@ -302,14 +302,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const bool need_mask = (CAUSAL && kv0 + 127 > q0 + t * 128 + p.off) || (kv0 + 128 > p.N_kv);
         if (need_mask) {
           const int lim = CAUSAL ? min(q_row + 1 + p.off, p.N_kv) : p.N_kv;  // keys [0, lim)
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < 128; ++c)
             if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
         }
-        float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
-        float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
-  #pragma unroll
-        for (int c = 4; c < 128; c += 8) {
+        // columns 0-7 seed the four running maxima; the loop takes 8 columns per step up to 127
+        float mx0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[4]));
+        float mx1 = fmaxf(__uint_as_float(s[1]), __uint_as_float(s[5]));
+        float mx2 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[6]));
+        float mx3 = fmaxf(__uint_as_float(s[3]), __uint_as_float(s[7]));
+#pragma unroll
+        for (int c = 8; c < 128; c += 8) {
           mx0 = max3f(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
           mx1 = max3f(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
           mx2 = max3f(mx2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         uint64_t lsum[4] = {0, 0, 0, 0}, rsum[4] = {0, 0, 0, 0};  // (0.f, 0.f) pairs
         uint32_t pk[64];
         if constexpr (!DROPOUT) {
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < 128; c += 2) {
             float a0, a1;
             f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, nbx2), a0, a1);
@@ -345,17 +348,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // kept ones (the keep scale is applied with 1/lr in the epilogue). Keys are taken 16
           // at a time: the quad's four lanes each run one generator call (one 4 x 4 block) and
           // swap words so that each lane holds its own row's bytes for the 16 keys.
-  #pragma unroll
+#pragma unroll
           for (int mc = 0; mc < 8; ++mc) {
             uint32_t kw[4] = {static_cast<uint32_t>(32 * j + 4 * mc + (lane & 3)),
                               static_cast<uint32_t>(q_row) >> 2, static_cast<uint32_t>(bh),
                               p.drop.offset};
             philox4x32_10(kw, p.drop.seed_lo, p.drop.seed_hi);
             quad_transpose(kw, lane);  // kw[g]: bytes of keys 16 mc + 4 g + (0..3), this row
-  #pragma unroll
+#pragma unroll
             for (int g = 0; g < 4; ++g) {
               const uint32_t kb = keep_bytes(kw[g], p.drop.add4);
-  #pragma unroll
+#pragma unroll
               for (int h = 0; h < 2; ++h) {
                 const int c = 16 * mc + 4 * g + 2 * h;
                 float a0, a1;
@@ -385,14 +388,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // only after the arrive below.
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
           const uint32_t tO = tmem + 256 + t * D + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < D; c += 32) {
             uint32_t o[32];
             tmem_ld_32x32b_x32(tO + c, o);
             tmem_ld_wait();
             reg_fence(o);
             const uint64_t a2 = f2_pack(alpha, alpha);
-  #pragma unroll
+#pragma unroll
             for (int i = 0; i < 32; i += 2) {
               const uint64_t r = f2_mul(f2_pack_u(o[i], o[i + 1]), a2);
               o[i] = static_cast<uint32_t>(r);

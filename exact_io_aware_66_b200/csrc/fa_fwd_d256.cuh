@@ -158,10 +158,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
         }
-        float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
-        float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
+        // columns 0-7 seed the four running maxima; the loop takes 8 columns per step up to 127
+        float mx0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[4]));
+        float mx1 = fmaxf(__uint_as_float(s[1]), __uint_as_float(s[5]));
+        float mx2 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[6]));
+        float mx3 = fmaxf(__uint_as_float(s[3]), __uint_as_float(s[7]));
 #pragma unroll
-        for (int c = 4; c < 128; c += 8) {
+        for (int c = 8; c < 128; c += 8) {
           mx0 = max3f(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
           mx1 = max3f(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
           mx2 = max3f(mx2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));

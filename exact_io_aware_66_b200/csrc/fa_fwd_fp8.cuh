@@ -232,14 +232,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const bool need_mask = (CAUSAL && kv0 + 127 > q0 + t * 128 + p.off) || (kv0 + 128 > p.N_kv);
         if (need_mask) {
           const int lim = CAUSAL ? min(q_row + 1 + p.off, p.N_kv) : p.N_kv;
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < 128; ++c)
             if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
         }
-        float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
-        float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
-  #pragma unroll
-        for (int c = 4; c < 128; c += 8) {
+        // columns 0-7 seed the four running maxima; the loop takes 8 columns per step up to 127
+        float mx0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[4]));
+        float mx1 = fmaxf(__uint_as_float(s[1]), __uint_as_float(s[5]));
+        float mx2 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[6]));
+        float mx3 = fmaxf(__uint_as_float(s[3]), __uint_as_float(s[7]));
+#pragma unroll
+        for (int c = 8; c < 128; c += 8) {
           mx0 = max3f(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
           mx1 = max3f(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
           mx2 = max3f(mx2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
@@ -257,7 +260,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint64_t sl2x2 = f2_pack(sl2, sl2), nbx2 = f2_pack(nb, nb);
         uint64_t lsum[2] = {0, 0}, rsum[2] = {0, 0};
         uint32_t pk[32];
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < 128; c += 4) {
           float a0, a1, a2, a3;
           f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, nbx2), a0, a1);
@@ -285,14 +288,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // O correction (PV(j-1) has completed: S(j) was issued after it).
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
           const uint32_t tO = tmem + 256 + t * 128 + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < 128; c += 32) {
             uint32_t o[32];
             tmem_ld_32x32b_x32(tO + c, o);
             tmem_ld_wait();
             reg_fence(o);
             const uint64_t a2 = f2_pack(alpha, alpha);
-  #pragma unroll
+#pragma unroll
             for (int i = 0; i < 32; i += 2) {
               const uint64_t r = f2_mul(f2_pack_u(o[i], o[i + 1]), a2);
               o[i] = static_cast<uint32_t>(r);
