@@ -348,6 +348,7 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   float* dq_acc = reinterpret_cast<float*>(ws);
   float* Dvec = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_D(BH, N, s.d));
   float* lse2 = reinterpret_cast<float*>(ws + fa::bwd_ws_offset_lse2(BH, N, s.d));
+  int* sched = reinterpret_cast<int*>(ws + fa::bwd_ws_offset_sched(BH, N, s.d));
   const int n64 = static_cast<int>(fa::bwd_n64(N));
   const long long rows = 1LL * BH * N;
 
@@ -382,11 +383,11 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
     if (s.d == 96)
       fa::fa_bwd_preprocess<96><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc, Dvec,
                                                                      lse2, rows, N, n64,
-        nullptr);
+        sched);
     else
       fa::fa_bwd_preprocess<D><<<nb, fa::kPrepThreads, 0, stream>>>(o16, do16, lse, dq_acc, Dvec,
                                                                     lse2, rows, N, n64,
-        nullptr);
+        sched);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd preprocess launch");
@@ -413,12 +414,17 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
   p.scale_log2 = s.scale * 1.4426950408889634f;
   p.drop = s.drop;
   apply_stall(2, p);
-  const long long grid = 1LL * p.n_kv * BHkv;
-  if (grid >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  // persistent: one CTA per SM (at most one per unit), units handed out by the counter
+  const long long units = 1LL * p.n_kv * BHkv;
+  if (units >= (1LL << 31)) return set_err(FA_ERR_UNSUPPORTED, "grid too large");
+  p.n_units = static_cast<int>(units);
+  p.sched_counter = sched;
+  const int n_sm = ds->n_sm > 0 ? ds->n_sm : 148;
+  const unsigned grid = static_cast<unsigned>(units < n_sm ? units : n_sm);
   {
     ProfileScope prof(2, stream);
-    kern<<<static_cast<unsigned>(grid), fa::kBwdThreads, L::kAlloc, stream>>>(
-        tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv, p);
+    kern<<<grid, fa::kBwdThreads, L::kAlloc, stream>>>(tq, tk, tv, tdo, tl, tD, tacc, tdk, tdv,
+                                                        p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "fa_bwd main launch");

@@ -10,8 +10,9 @@
 //
 // Three kernels run in order on the caller's stream:
 //   1. fa_bwd_preprocess: D = rowsum(dO o O) (fp32), lse2 = -lse * log2(e), dQ_acc = 0.
-//   2. fa_bwd_main: one CTA per (key/value head, 128-key tile j), looping over every query
-//      head that shares the key/value head and over the 64-row query tiles that see tile j.
+//   2. fa_bwd_main: a persistent kernel whose work units are (key/value head, 128-key tile j),
+//      each looping over every query head that shares the key/value head and over the 64-row
+//      query tiles that see tile j (one CTA per SM takes units from a counter).
 //      K_j and V_j stay in shared memory; tiles of Q and dO stream through a 3-stage TMA ring
 //      (4 at d = 64). Per query tile i, five tcgen05 MMAs (all M = 128):
 //          S^T  = K_j Q_i^T          -> TMEM (64 columns, double buffered)
@@ -22,7 +23,8 @@
 //      Two warpgroups turn S^T/dP^T into P^T (back to TMEM) and dS^T (to shared memory) while
 //      the tensor core works on the previous tile; a third drains dQ^T from TMEM and adds it
 //      into the fp32 accumulator with TMA bulk reductions (cp.reduce.async.bulk .add.f32).
-//      The final dK (times scale) and dV are stored with TMA. With dropout (DROPOUT), the
+//      The final dK (times scale) and dV are stored with TMA by the drain warps, while the
+//      others start the next unit. With dropout (DROPOUT), the
 //      elementwise warps regenerate the keep decisions of the forward (dropout.cuh) and form
 //      dS = P o (r Z o dP - D) and Z o P for the dV product; dV is scaled by r at the end.
 //   3. fa_bwd_dq_convert: dQ = bf16(dQ_acc).
@@ -147,9 +149,14 @@ struct BwdLayout {
   static constexpr int bDSFree = bSdPFull + 8;          // + buffer
   static constexpr int bAccDone = bSdPFull + 10;
   static constexpr int bDrain = bSdPFull + 11;
-  static constexpr int kNumBars = bDrain + 1;
+  static constexpr int bAccFree = bSdPFull + 12;        // dV, dK of the unit read out (128)
+  static constexpr int bSchedFull = bSdPFull + 13;      // + slot: next unit index published
+  static constexpr int bSchedEmpty = bSdPFull + 15;     // + slot: read by every consuming warp
+  static constexpr int kNumBars = bSdPFull + 17;
+  static constexpr int kSchedReaders = 13;              // warps 0-11 and the MMA thread
 
-  static constexpr int kTmemSlot = kBars + kNumBars * 8;
+  static constexpr int kSched = kBars + kNumBars * 8;  // two unit indices (-1: no unit left)
+  static constexpr int kTmemSlot = kSched + 8;
   static constexpr int kBytes = kTmemSlot + 16;
   static constexpr int kAlloc = kBytes + 1024;
 
@@ -159,6 +166,8 @@ struct BwdLayout {
   __host__ __device__ static constexpr uint32_t tS(int b) { return 256u + 128u * b; }
   __host__ __device__ static constexpr uint32_t tDP(int b) { return 256u + 128u * b + 64u; }
 };
+// (plus the kernel's few bytes of static shared memory)
+static_assert(BwdLayout<128>::kAlloc + 16 <= 227 * 1024, "64-row backward shared memory");
 
 struct BwdParams {
   int* status;
@@ -205,20 +214,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Heads are processed in groups of p.group, sized on the host so that a group's Q, dO, K, V
-  // and dQ accumulator fit in L2; within a group the key tiles with the most query tiles
-  // (causal) come first, cycling over the group's heads (longest-processing-time order).
   constexpr int QS = L::kQStages;
-  int j, bh;  // key tile, key/value head
-  grouped_unit(static_cast<int>(blockIdx.x), p.n_kv, p.BH_kv, p.group, j, bh);
-  const int k0 = 128 * j;
-  // First 64-row query tile with a query that sees a key of this tile (j <= i + off), and the
-  // iterations: every query head that shares this key/value head, times its query tiles.
-  const int qi0 = CAUSAL ? max(0, k0 - p.off) / 64 : 0;
-  const int n_qt = max(0, p.n_q - qi0);
-  const int n_i = p.qgroup * n_qt;
-  auto q_head = [&](int it) { return bh * p.qgroup + it / n_qt; };
-  auto q_tile = [&](int it) { return qi0 + it % n_qt; };
+  // The kernel is persistent: one CTA per SM (at most one per unit) takes work units — one
+  // (key/value head, 128-key tile j) each — unit blockIdx.x first, then gridDim.x + the value
+  // of a counter in the workspace (zeroed by the preprocess kernel), in the order of
+  // grouped_unit: groups of p.group heads sized so that a group's Q, dO, K, V and dQ
+  // accumulator fit in L2, the key tiles with the most query tiles first inside a group. A
+  // unit loops over every query head that shares its key/value head and over the 64-row query
+  // tiles that see its keys. Every pipeline barrier counts its phases over the CTA's run.
+  struct Unit {
+    int bh, k0, qi0, n_qt, n_i;
+  };
+  auto unit_of = [&](int u) {
+    Unit w;
+    int j;
+    grouped_unit(u, p.n_kv, p.BH_kv, p.group, j, w.bh);
+    w.k0 = 128 * j;
+    // first 64-row query tile with a query that sees a key of this tile (j <= i + off)
+    w.qi0 = CAUSAL ? max(0, w.k0 - p.off) / 64 : 0;
+    w.n_qt = max(0, p.n_q - w.qi0);
+    w.n_i = p.qgroup * w.n_qt;
+    return w;
+  };
+  volatile int* sched = reinterpret_cast<volatile int*>(gbase + L::kSched);
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -233,8 +251,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(L::bDQFull + s), 1);
       mbar_init(bar(L::bDQFree + s), 128);
       mbar_init(bar(L::bDSFree + s), 1);
+      mbar_init(bar(L::bSchedFull + s), 1);
+      mbar_init(bar(L::bSchedEmpty + s), L::kSchedReaders);
     }
     mbar_init(bar(L::bAccDone), 1);
+    mbar_init(bar(L::bAccFree), 128);
     mbar_init(bar(L::bDrain), 1);
     fence_barrier_init();
   }
@@ -254,190 +275,238 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::kTmemSlot);
 
+  // Unit number s of this CTA, as a whole warp: wait for the TMA thread to publish it, then
+  // acknowledge the read (one arrival per warp). -1: no unit left; kGaveUp: the wait gave up.
+  constexpr int kGaveUp = -2;
+  auto warp_next_unit = [&](int s) -> int {
+    if (!warp_wait(bar(L::bSchedFull + (s & 1)), (s >> 1) & 1, abort_flag)) return kGaveUp;
+    const int u = sched[s & 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::bSchedEmpty + (s & 1)));
+    return u;
+  };
+
   if (warp < 8) {
     // ------------------------------------------------------- P^T and dS^T (elementwise) ---
     const int w = warp >> 2;                       // query columns [32w, 32w+32)
     const int r = threadIdx.x & 127;               // key row within the tile (TMEM lane)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int key = k0 + r;
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int i = 0; i < n_i && ok; ++i) {
-      const int b = i & 1, st = i % QS;
-      const int qi = q_tile(i);
-      ok = warp_wait(bar(L::bQFull + st), (i / QS) & 1, abort_flag) &&
-           warp_wait(bar(L::bSdPFull + b), (i >> 1) & 1, abort_flag) &&
-           (i < 2 || warp_wait(bar(L::bDSFree + b), ((i >> 1) & 1) ^ 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t s[32], dp[32];
-      tmem_ld_32x32b_x32(tmem + L::tS(b) + 32 * w + lane_off, s);
-      tmem_ld_32x32b_x32(tmem + L::tDP(b) + 32 * w + lane_off, dp);
-      tmem_ld_wait();
-      reg_fence(s);
-      reg_fence(dp);
-      const float* lse2 = reinterpret_cast<const float*>(gbase + L::kRow + st * 512) + 32 * w;
-      const float* Dv = reinterpret_cast<const float*>(gbase + L::kRow + st * 512 + 256) + 32 * w;
-      const int qbase = 64 * qi + 32 * w;
-      const bool need_mask = (CAUSAL && qbase + p.off < k0 + 127) || (qbase + 32 > p.N) ||
-                             (k0 + 128 > p.N_kv);
-      uint32_t pk[16], dsk[16];
-      const uint64_t sl2x2 = f2_pack(sl2, sl2);
-      // Dropout keep bits of this key for the 32 queries: the quad's four lanes (keys 4J..4J+3)
-      // run two generator calls each (blocks of queries 4n..4n+3 for n = lane%4 and 4 + lane%4),
-      // transpose each block's bytes so that word t holds key t's four bytes, and swap words:
-      // kbits[h][g] then holds queries qbase + 16h + 4g + (0..3) of this key.
-      uint32_t kbits[2][4];
-      if constexpr (DROPOUT) {
+    int g = 0;  // tiles of this CTA's earlier units
+    for (int si = 0; ok; ++si) {
+      const int u = warp_next_unit(si);
+      if (u == kGaveUp) { ok = false; break; }
+      if (u < 0) break;
+      const Unit U = unit_of(u);
+      const int key = U.k0 + r;
+      for (int i = 0; i < U.n_i && ok; ++i, ++g) {
+        const int b = g & 1, st = g % QS;
+        const int qi = U.qi0 + i % U.n_qt, qh = U.bh * p.qgroup + i / U.n_qt;
+        ok = warp_wait(bar(L::bQFull + st), (g / QS) & 1, abort_flag) &&
+             warp_wait(bar(L::bSdPFull + b), (g >> 1) & 1, abort_flag) &&
+             (g < 2 || warp_wait(bar(L::bDSFree + b), ((g >> 1) & 1) ^ 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t s[32], dp[32];
+        tmem_ld_32x32b_x32(tmem + L::tS(b) + 32 * w + lane_off, s);
+        tmem_ld_32x32b_x32(tmem + L::tDP(b) + 32 * w + lane_off, dp);
+        tmem_ld_wait();
+        reg_fence(s);
+        reg_fence(dp);
+        const float* lse2 = reinterpret_cast<const float*>(gbase + L::kRow + st * 512) + 32 * w;
+        const float* Dv =
+            reinterpret_cast<const float*>(gbase + L::kRow + st * 512 + 256) + 32 * w;
+        const int qbase = 64 * qi + 32 * w;
+        const bool need_mask = (CAUSAL && qbase + p.off < U.k0 + 127) || (qbase + 32 > p.N) ||
+                               (U.k0 + 128 > p.N_kv);
+        uint32_t pk[16], dsk[16];
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        // Dropout keep bits of this key for the 32 queries: the quad's four lanes (keys 4J..4J+3)
+        // run two generator calls each (blocks of queries 4n..4n+3 for n = lane%4 and 4 + lane%4),
+        // transpose each block's bytes so that word t holds key t's four bytes, and swap words:
+        // kbits[h][g] then holds queries qbase + 16h + 4g + (0..3) of this key.
+        uint32_t kbits[2][4];
+        if constexpr (DROPOUT) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t wv[4] = {static_cast<uint32_t>(key) >> 2,
-                            static_cast<uint32_t>((qbase >> 2) + 4 * h + (lane & 3)),
-                            static_cast<uint32_t>(q_head(i)), p.drop.offset};
-          philox4x32_10(wv, p.drop.seed_lo, p.drop.seed_hi);
-          byte_transpose(wv, kbits[h]);
-          quad_transpose(kbits[h], lane);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t wv[4] = {static_cast<uint32_t>(key) >> 2,
+                              static_cast<uint32_t>((qbase >> 2) + 4 * h + (lane & 3)),
+                              static_cast<uint32_t>(qh), p.drop.offset};
+            philox4x32_10(wv, p.drop.seed_lo, p.drop.seed_hi);
+            byte_transpose(wv, kbits[h]);
+            quad_transpose(kbits[h], lane);
 #pragma unroll
-          for (int g = 0; g < 4; ++g) kbits[h][g] = keep_bytes(kbits[h][g], p.drop.add4);
-        }
-      }
-      const uint64_t rk2 = f2_pack(p.drop.keep_scale, p.drop.keep_scale);
-#pragma unroll
-      for (int c = 0; c < 32; c += 4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);  // -lse * log2(e)
-        const float4 d4 = *reinterpret_cast<const float4*>(Dv + c);
-        float a[4], pr[4], dsr[4];
-        f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, f2_pack(l4.x, l4.y)), a[0], a[1]);
-        f2_unpack(f2_fma(f2_pack_u(s[c + 2], s[c + 3]), sl2x2, f2_pack(l4.z, l4.w)), a[2], a[3]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) pr[e] = ex2_approx(a[e]);
-        if constexpr (!DROPOUT) {
-          f2_unpack(f2_mul(f2_pack(pr[0], pr[1]),
-                           f2_sub(f2_pack_u(dp[c], dp[c + 1]), f2_pack(d4.x, d4.y))),
-                    dsr[0], dsr[1]);
-          f2_unpack(f2_mul(f2_pack(pr[2], pr[3]),
-                           f2_sub(f2_pack_u(dp[c + 2], dp[c + 3]), f2_pack(d4.z, d4.w))),
-                    dsr[2], dsr[3]);
-        } else {
-          // dS = P o (r Z o dP - D); the P fed to the dV MMA is Z o P (r is applied to dV at
-          // the end)
-          const uint32_t kb = kbits[c / 16][(c / 4) & 3];
-          const uint32_t m0 = elem_mask<0>(kb), m1 = elem_mask<1>(kb);
-          const uint32_t m2 = elem_mask<2>(kb), m3 = elem_mask<3>(kb);
-          f2_unpack(f2_mul(f2_pack(pr[0], pr[1]),
-                           f2_fma(f2_pack_u(dp[c] & m0, dp[c + 1] & m1), rk2,
-                                  f2_pack(-d4.x, -d4.y))),
-                    dsr[0], dsr[1]);
-          f2_unpack(f2_mul(f2_pack(pr[2], pr[3]),
-                           f2_fma(f2_pack_u(dp[c + 2] & m2, dp[c + 3] & m3), rk2,
-                                  f2_pack(-d4.z, -d4.w))),
-                    dsr[2], dsr[3]);
-          pr[0] = __uint_as_float(__float_as_uint(pr[0]) & m0);
-          pr[1] = __uint_as_float(__float_as_uint(pr[1]) & m1);
-          pr[2] = __uint_as_float(__float_as_uint(pr[2]) & m2);
-          pr[3] = __uint_as_float(__float_as_uint(pr[3]) & m3);
-        }
-        if (need_mask) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int q = qbase + c + e;
-            if (q >= p.N || key >= p.N_kv || (CAUSAL && q + p.off < key)) {
-              pr[e] = 0.f;
-              dsr[e] = 0.f;
-            }
+            for (int g = 0; g < 4; ++g) kbits[h][g] = keep_bytes(kbits[h][g], p.drop.add4);
           }
         }
-        pk[c / 2] = pack_bf16x2(pr[0], pr[1]);
-        pk[c / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
-        dsk[c / 2] = pack_bf16x2(dsr[0], dsr[1]);
-        dsk[c / 2 + 1] = pack_bf16x2(dsr[2], dsr[3]);
-      }
-      tmem_st_32x32b_x16(tmem + L::tS(b) + 32 * w + lane_off, pk);
-      uint8_t* dsb = gbase + L::kDS + b * 16384;
+        const uint64_t rk2 = f2_pack(p.drop.keep_scale, p.drop.keep_scale);
 #pragma unroll
-      for (int t = 0; t < 4; ++t)
-        *reinterpret_cast<uint4*>(dsb + sw128_offset(r, 4 * w + t)) =
-            make_uint4(dsk[4 * t], dsk[4 * t + 1], dsk[4 * t + 2], dsk[4 * t + 3]);
-      tmem_st_wait();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(L::bEwDone + b));
+        for (int c = 0; c < 32; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);  // -lse * log2(e)
+          const float4 d4 = *reinterpret_cast<const float4*>(Dv + c);
+          float a[4], pr[4], dsr[4];
+          f2_unpack(f2_fma(f2_pack_u(s[c], s[c + 1]), sl2x2, f2_pack(l4.x, l4.y)), a[0], a[1]);
+          f2_unpack(f2_fma(f2_pack_u(s[c + 2], s[c + 3]), sl2x2, f2_pack(l4.z, l4.w)), a[2], a[3]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pr[e] = ex2_approx(a[e]);
+          if constexpr (!DROPOUT) {
+            f2_unpack(f2_mul(f2_pack(pr[0], pr[1]),
+                             f2_sub(f2_pack_u(dp[c], dp[c + 1]), f2_pack(d4.x, d4.y))),
+                      dsr[0], dsr[1]);
+            f2_unpack(f2_mul(f2_pack(pr[2], pr[3]),
+                             f2_sub(f2_pack_u(dp[c + 2], dp[c + 3]), f2_pack(d4.z, d4.w))),
+                      dsr[2], dsr[3]);
+          } else {
+            // dS = P o (r Z o dP - D); the P fed to the dV MMA is Z o P (r is applied to dV at
+            // the end)
+            const uint32_t kb = kbits[c / 16][(c / 4) & 3];
+            const uint32_t m0 = elem_mask<0>(kb), m1 = elem_mask<1>(kb);
+            const uint32_t m2 = elem_mask<2>(kb), m3 = elem_mask<3>(kb);
+            f2_unpack(f2_mul(f2_pack(pr[0], pr[1]),
+                             f2_fma(f2_pack_u(dp[c] & m0, dp[c + 1] & m1), rk2,
+                                    f2_pack(-d4.x, -d4.y))),
+                      dsr[0], dsr[1]);
+            f2_unpack(f2_mul(f2_pack(pr[2], pr[3]),
+                             f2_fma(f2_pack_u(dp[c + 2] & m2, dp[c + 3] & m3), rk2,
+                                    f2_pack(-d4.z, -d4.w))),
+                      dsr[2], dsr[3]);
+            pr[0] = __uint_as_float(__float_as_uint(pr[0]) & m0);
+            pr[1] = __uint_as_float(__float_as_uint(pr[1]) & m1);
+            pr[2] = __uint_as_float(__float_as_uint(pr[2]) & m2);
+            pr[3] = __uint_as_float(__float_as_uint(pr[3]) & m3);
+          }
+          if (need_mask) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int q = qbase + c + e;
+              if (q >= p.N || key >= p.N_kv || (CAUSAL && q + p.off < key)) {
+                pr[e] = 0.f;
+                dsr[e] = 0.f;
+              }
+            }
+          }
+          pk[c / 2] = pack_bf16x2(pr[0], pr[1]);
+          pk[c / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
+          dsk[c / 2] = pack_bf16x2(dsr[0], dsr[1]);
+          dsk[c / 2 + 1] = pack_bf16x2(dsr[2], dsr[3]);
+        }
+        tmem_st_32x32b_x16(tmem + L::tS(b) + 32 * w + lane_off, pk);
+        uint8_t* dsb = gbase + L::kDS + b * 16384;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          *reinterpret_cast<uint4*>(dsb + sw128_offset(r, 4 * w + t)) =
+              make_uint4(dsk[4 * t], dsk[4 * t + 1], dsk[4 * t + 2], dsk[4 * t + 3]);
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(L::bEwDone + b));
+      }
     }
     if (!ok) fail(p.status, abort_flag, 5);
-    // ------------------------------------------------------------ dV / dK epilogue -------
-    if (ok && (n_i == 0 || warp_wait(bar(L::bAccDone), 0, abort_flag))) {
-      tc_fence_after();
-      // warpgroup 0 stores dV (stage-0 Q/dO space), warpgroup 1 stores dK * scale (stage 1)
-      const uint32_t tcol = w == 0 ? L::tDV : L::tDK;
-      const float mul = w == 0 ? (DROPOUT ? p.drop.keep_scale : 1.0f) : p.scale;
-      const int region = L::kQ + w * 2 * L::kQTile;
-      uint8_t* stage = gbase + region;
-#pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        uint32_t v[32];
-        if (n_i > 0) {
-          tmem_ld_32x32b_x32(tmem + tcol + c + lane_off, v);
-          tmem_ld_wait();
-          reg_fence(v);
-        } else {  // no query sees these keys: dK = dV = 0 (TMEM was never written)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0u;
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * mul, __uint_as_float(v[8 * q + 1]) * mul);
-          u.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * mul, __uint_as_float(v[8 * q + 3]) * mul);
-          u.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * mul, __uint_as_float(v[8 * q + 5]) * mul);
-          u.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * mul, __uint_as_float(v[8 * q + 7]) * mul);
-          const int chunk = c / 8 + q;
-          *reinterpret_cast<uint4*>(stage + (chunk >> 3) * L::kKVBox + sw128_offset(r, chunk & 7)) = u;
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        const CUtensorMap* map = w == 0 ? &tmDV : &tmDK;
-#pragma unroll
-        for (int bx = 0; bx < L::kBoxes; ++bx)
-          tma_store_3d(map, sbase + region + bx * L::kKVBox + (warp & 3) * 4096, 64 * bx,
-                       k0 + (warp & 3) * 32, bh);
-        bulk_commit_group();
-        bulk_wait_group_read0();
-      }
-    } else if (ok) {
-      fail(p.status, abort_flag, 5);
-    }
   } else if (warp < 12) {
-    // ---------------------------------------------------------------- dQ drain ----------
+    // ------------------------------------------ dQ drain, and the unit's dK / dV -----------
     const int wq = warp & 3;                         // d columns [32 wq, 32 wq + 32)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     float* stagef = reinterpret_cast<float*>(gbase + L::kDQ + wq * 8192);
+    uint8_t* stageb = gbase + L::kDQ + wq * 8192;
     const uint32_t stage_s = sbase + L::kDQ + wq * 8192;
     const bool active = 32 * wq < p.d;
+    const float scale = p.scale;
+    const float dv_mul = DROPOUT ? p.drop.keep_scale : 1.0f;  // dV = r (Z o P)^T dO
     bool ok = true;
-    for (int i = 0; i < n_i; ++i) {
-      const int b = i & 1;
-      if (!warp_wait(bar(L::bDQFull + b), (i >> 1) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t v[64];
-      tmem_ld_32x32b_x32(tmem + L::tDP(b) + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld_32x32b_x32(tmem + L::tDP(b) + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-      tmem_ld_wait();
-      reg_fence(v);
-      tc_fence_before();
-      mbar_arrive(bar(L::bDQFree + b));
-      if (!active) continue;
-      if (lane == 0) bulk_wait_group_read0();  // previous reduction finished reading staging
-      __syncwarp();
+    int g = 0, uc = 0;  // tiles of earlier units; earlier units with at least one tile
+    for (int si = 0; ok; ++si) {
+      const int u = warp_next_unit(si);
+      if (u == kGaveUp) { ok = false; break; }
+      if (u < 0) break;
+      const Unit U = unit_of(u);
+      for (int i = 0; i < U.n_i; ++i, ++g) {
+        const int b = g & 1;
+        if (!warp_wait(bar(L::bDQFull + b), (g >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[64];
+        tmem_ld_32x32b_x32(tmem + L::tDP(b) + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld_32x32b_x32(tmem + L::tDP(b) + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld_wait();
+        reg_fence(v);
+        tc_fence_before();
+        mbar_arrive(bar(L::bDQFree + b));
+        if (!active) continue;
+        const int qi = U.qi0 + i % U.n_qt, qh = U.bh * p.qgroup + i / U.n_qt;
+        if (lane == 0) bulk_wait_group_read0();  // previous bulk copy finished reading staging
+        __syncwarp();
 #pragma unroll
-      for (int q = 0; q < 64; ++q) stagef[q * 32 + lane] = __uint_as_float(v[q]) * p.scale;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_reduce_add_3d(&tmDQacc, stage_s, 32 * wq, 64 * q_tile(i), q_head(i));
-        bulk_commit_group();
+        for (int q = 0; q < 64; ++q) stagef[q * 32 + lane] = __uint_as_float(v[q]) * scale;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tmDQacc, stage_s, 32 * wq, 64 * qi, qh);
+          bulk_commit_group();
+        }
       }
+      if (!ok) break;
+      // dV and dK * scale of the unit (zero when no query sees its keys): TMEM -> bf16 ->
+      // staging (32 rows x 64 columns per 4 KB box, 128-byte swizzle) -> TMA store; at d = 128
+      // dK reuses dV's staging once dV's store has read it, and TMEM is released after dK.
+      const bool has = U.n_i > 0;
+      if (has) {
+        if (!warp_wait(bar(L::bAccDone), uc & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+      }
+      const int row0 = U.k0 + 32 * wq;
+      // one accumulator (TMEM columns tcol) times mul into the staging at byte offset soff
+      auto stage_acc = [&](uint32_t tcol, float mul, int soff) {
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t v[32];
+          if (has) {
+            tmem_ld_32x32b_x32(tmem + tcol + c + lane_off, v);
+            tmem_ld_wait();
+            reg_fence(v);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = c / 8 + q;
+            *reinterpret_cast<uint4*>(stageb + soff + (chunk >> 3) * 4096 +
+                                      sw128_offset(lane, chunk & 7)) =
+                make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]) * mul, __uint_as_float(v[8 * q + 1]) * mul),
+                           pack_bf16x2(__uint_as_float(v[8 * q + 2]) * mul, __uint_as_float(v[8 * q + 3]) * mul),
+                           pack_bf16x2(__uint_as_float(v[8 * q + 4]) * mul, __uint_as_float(v[8 * q + 5]) * mul),
+                           pack_bf16x2(__uint_as_float(v[8 * q + 6]) * mul, __uint_as_float(v[8 * q + 7]) * mul));
+          }
+        }
+      };
+      auto store_acc = [&](const CUtensorMap* map, int soff) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int bx = 0; bx < L::kBoxes; ++bx)
+            tma_store_3d(map, stage_s + soff + bx * 4096, 64 * bx, row0, U.bh);
+          bulk_commit_group();
+        }
+      };
+      // at d = 64 dV and dK sit side by side in the 8 KB; at d = 128 dK reuses dV's space
+      constexpr int kDKOff = D == 64 ? 4096 : 0;
+      if (lane == 0) bulk_wait_group_read0();
+      __syncwarp();
+      stage_acc(L::tDV, dv_mul, 0);
+      store_acc(&tmDV, 0);
+      if constexpr (D == 128) {
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+      }
+      stage_acc(L::tDK, scale, kDKOff);
+      if (has) {
+        tc_fence_before();
+        mbar_arrive(bar(L::bAccFree));
+        ++uc;
+      }
+      store_acc(&tmDK, kDKOff);
     }
     if (!ok) fail(p.status, abort_flag, 5);
     if (lane == 0) bulk_wait_group0();
@@ -478,12 +547,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         umma_commit(bar(L::bSdPFull + b));
       };
-      auto second_half = [&](int i) {
+      auto second_half = [&](int i, bool acc_prev) {
         const int b = i & 1, st = i % QS;
         const uint32_t so = static_cast<uint32_t>(st) * 2 * L::kQTile;
         const uint64_t qmn = sdesc_advance(dQ_mn, so), omn = sdesc_advance(dDO_mn, so);
         const uint64_t ds = sdesc_advance(dDS, b * 16384);
-        const uint32_t acc = i > 0 ? 1u : 0u;
+        const uint32_t acc = acc_prev ? 1u : 0u;  // dV, dK accumulate after the unit's first
         // dV += P^T dO: P^T (keys x 64 queries) from TMEM; query columns 0-31 were packed into
         // S columns [0,16), 32-63 into [32,48).
 #pragma unroll
@@ -506,29 +575,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         umma_commit(bar(L::bDSFree + b));
       };
       const uint64_t lim = p.limit_ns;
-      bool ok = n_i == 0 || mbar_wait(bar(L::bKV), 0, abort_flag, lim);
-      for (int i = 0; i < n_i && ok; ++i) {
-        const int b = i & 1, st = i % QS;
-        ok = mbar_wait(bar(L::bQFull + st), (i / QS) & 1, abort_flag, lim) &&
-             (i < 2 || mbar_wait(bar(L::bDQFree + b), ((i >> 1) & 1) ^ 1, abort_flag, lim));
+      bool ok = true;
+      int g = 0, uc = 0;  // tiles of earlier units; earlier units with at least one tile
+      for (int si = 0; ok; ++si) {
+        if (!(ok = mbar_wait(bar(L::bSchedFull + (si & 1)), (si >> 1) & 1, abort_flag, lim))) break;
+        const int u = sched[si & 1];
+        mbar_arrive(bar(L::bSchedEmpty + (si & 1)));
+        if (u < 0) break;
+        const int n_i = unit_of(u).n_i;
+        if (n_i == 0) continue;
+        if (!(ok = mbar_wait(bar(L::bKV), uc & 1, abort_flag, lim))) break;
+        // the unit's first dV/dK products overwrite TMEM the previous unit's epilogue reads
+        auto second = [&](int i) -> bool {
+          const int gi = g + i;
+          if (!mbar_wait(bar(L::bEwDone + (gi & 1)), (gi >> 1) & 1, abort_flag, lim)) return false;
+          if (i == 0 && uc > 0 && !mbar_wait(bar(L::bAccFree), (uc - 1) & 1, abort_flag, lim))
+            return false;
+          tc_fence_after();
+          second_half(gi, i > 0);
+          return true;
+        };
+        for (int i = 0; i < n_i && ok; ++i) {
+          const int gi = g + i, b = gi & 1, st = gi % QS;
+          ok = mbar_wait(bar(L::bQFull + st), (gi / QS) & 1, abort_flag, lim) &&
+               (gi < 2 || mbar_wait(bar(L::bDQFree + b), ((gi >> 1) & 1) ^ 1, abort_flag, lim));
+          if (!ok) break;
+          tc_fence_after();
+          first_half(gi);
+          if (i > 0) ok = second(i - 1);
+        }
+        if (ok) ok = second(n_i - 1);
         if (!ok) break;
-        tc_fence_after();
-        first_half(i);
-        if (i > 0) {
-          const int pb = (i - 1) & 1;
-          if (!mbar_wait(bar(L::bEwDone + pb), ((i - 1) >> 1) & 1, abort_flag, lim)) { ok = false; break; }
-          tc_fence_after();
-          second_half(i - 1);
-        }
-      }
-      if (ok && n_i > 0) {
-        const int i = n_i - 1;
-        ok = mbar_wait(bar(L::bEwDone + (i & 1)), (i >> 1) & 1, abort_flag, lim);
-        if (ok) {
-          tc_fence_after();
-          second_half(i);
-          umma_commit(bar(L::bAccDone));
-        }
+        umma_commit(bar(L::bAccDone));
+        g += n_i;
+        ++uc;
       }
       if (!ok) fail(p.status, abort_flag, 5);
       // Every MMA this thread issued completes before tensor memory is freed (the drain after a
@@ -538,44 +618,75 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait(bar(L::bDrain), 0, &never);
     }
   } else if (warp == 13) {
-    // --------------------------------------------------------------------- TMA ----------
+    // ---------------------------------------------------- TMA, and the unit scheduler -----
     if (lane == 0) {
-      if (n_i > 0) {
-        mbar_arrive_expect_tx(bar(L::bKV), 2 * L::kKVTile);
-#pragma unroll
-        for (int bx = 0; bx < L::kBoxes; ++bx) {
-          tma_load_3d(sbase + L::kK + bx * L::kKVBox, &tmK, bar(L::bKV), 64 * bx, k0, bh);
-          tma_load_3d(sbase + L::kV + bx * L::kKVBox, &tmV, bar(L::bKV), 64 * bx, k0, bh);
-        }
-      }
-      int issued = 0;
-      for (int i = 0; i < n_i; ++i) {
-        const int st = i % QS;
-        if (!mbar_wait(bar(L::bQEmpty + st), ((i / QS) & 1) ^ 1, abort_flag)) {
-          fail(p.status, abort_flag, 5);
+      bool ok = true;
+      int g = 0, uc = 0;
+      int issued = 0, skipped = -1, kv_loads = 0;
+      int u = static_cast<int>(blockIdx.x);
+      for (int si = 0;; ++si) {
+        // publish unit si of this CTA (-1 when none is left) once every reader took unit si-2
+        if (!mbar_wait(bar(L::bSchedEmpty + (si & 1)), ((si >> 1) & 1) ^ 1, abort_flag)) {
+          ok = false;
           break;
         }
-        const int q0 = 64 * q_tile(i), qh = q_head(i);
-        issued = i + 1;
-        if (i == p.dbg_skip) continue;  // (the test hook leaves this tile out)
-        mbar_arrive_expect_tx(bar(L::bQFull + st), 2 * L::kQTile + 512);
+        const int pub = u < p.n_units ? u : -1;
+        sched[si & 1] = pub;
+        mbar_arrive(bar(L::bSchedFull + (si & 1)));
+        if (pub < 0) break;
+        const Unit U = unit_of(u);
+        for (int i = 0; i < U.n_i; ++i) {
+          const int gi = g + i, st = gi % QS;
+          if (!mbar_wait(bar(L::bQEmpty + st), ((gi / QS) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int q0 = 64 * (U.qi0 + i % U.n_qt), qh = U.bh * p.qgroup + i / U.n_qt;
+          issued = gi + 1;
+          if (i == p.dbg_skip) {  // (the test hook leaves this tile out)
+            skipped = gi;
+          } else {
+            mbar_arrive_expect_tx(bar(L::bQFull + st), 2 * L::kQTile + 512);
 #pragma unroll
-        for (int bx = 0; bx < L::kBoxes; ++bx) {
-          tma_load_3d(sbase + L::kQ + st * 2 * L::kQTile + bx * L::kQBox, &tmQ,
-                      bar(L::bQFull + st), 64 * bx, q0, qh);
-          tma_load_3d(sbase + L::kDO + st * 2 * L::kQTile + bx * L::kQBox, &tmDO,
-                      bar(L::bQFull + st), 64 * bx, q0, qh);
+            for (int bx = 0; bx < L::kBoxes; ++bx) {
+              tma_load_3d(sbase + L::kQ + st * 2 * L::kQTile + bx * L::kQBox, &tmQ,
+                          bar(L::bQFull + st), 64 * bx, q0, qh);
+              tma_load_3d(sbase + L::kDO + st * 2 * L::kQTile + bx * L::kQBox, &tmDO,
+                          bar(L::bQFull + st), 64 * bx, q0, qh);
+            }
+            tma_load_3d(sbase + L::kRow + st * 512, &tmLse2, bar(L::bQFull + st), q0, qh, 0);
+            tma_load_3d(sbase + L::kRow + st * 512 + 256, &tmD, bar(L::bQFull + st), q0, qh, 0);
+          }
+          if (i == 0) {
+            // K and V of the unit, once every product of the previous unit has completed
+            if (uc > 0 && !mbar_wait(bar(L::bAccDone), (uc - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(L::bKV), 2 * L::kKVTile);
+#pragma unroll
+            for (int bx = 0; bx < L::kBoxes; ++bx) {
+              tma_load_3d(sbase + L::kK + bx * L::kKVBox, &tmK, bar(L::bKV), 64 * bx, U.k0, U.bh);
+              tma_load_3d(sbase + L::kV + bx * L::kKVBox, &tmV, bar(L::bKV), 64 * bx, U.k0, U.bh);
+            }
+            kv_loads = uc + 1;
+          }
         }
-        tma_load_3d(sbase + L::kRow + st * 512, &tmLse2, bar(L::bQFull + st), q0, qh, 0);
-        tma_load_3d(sbase + L::kRow + st * 512 + 256, &tmD, bar(L::bQFull + st), q0, qh, 0);
+        if (!ok) break;
+        if (U.n_i > 0) {
+          g += U.n_i;
+          ++uc;
+        }
+        u = static_cast<int>(gridDim.x) + atomicAdd(p.sched_counter, 1);
       }
+      if (!ok) fail(p.status, abort_flag, 5);
       // Every load issued lands before the CTA can exit, whether or not (or whenever) a role
       // gives up; the last QS loads are the latest in their stages, so on the normal path these
       // bounded waits return at once.
       volatile int never = 0;
       for (int i = max(0, issued - QS); i < issued; ++i)
-        if (i != p.dbg_skip) mbar_wait(bar(L::bQFull + (i % QS)), (i / QS) & 1, &never);
-      if (n_i > 0) mbar_wait(bar(L::bKV), 0, &never);
+        if (i != skipped) mbar_wait(bar(L::bQFull + (i % QS)), (i / QS) & 1, &never);
+      if (kv_loads > 0) mbar_wait(bar(L::bKV), (kv_loads - 1) & 1, &never);
     }
   }
   tc_fence_before();
