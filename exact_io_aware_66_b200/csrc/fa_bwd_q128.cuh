@@ -18,16 +18,18 @@
 //   * TMEM holds exactly four 128-column fp32 regions: dV, dK, S^T (then P^T in place) and dP^T
 //     (then dQ^T in place; at d = 64, dQ = dS K with the queries on the lanes, since an M = 64
 //     product would leave half the lanes idle). Nothing is double buffered; the MMA issue order is
-//         S(i), dK(i-1), dQ(i-1), dV(i), dP(i), S(i+1), ...
-//     so the elementwise warps turn S^T(i) into P^T(i) while the tensor core finishes tile i-1,
-//     and the dQ^T(i-1) drain overlaps dV(i).
+//         S(i), dK(i-1), dQ(i-1), dP(i), dV(i), S(i+1), ...
+//     so the elementwise warps turn S^T(i) into P^T(i) while the tensor core finishes tile i-1
+//     and computes dP^T(i) (which does not wait for P^T(i)). At d = 64, where the products are
+//     short, dP(i) and dV(i) go in whichever order their inputs arrive, so that dV(i) can fill
+//     the wait for the drain of dQ(i-1) when P^T(i) is ready first.
 //   * The drain warpgroup copies all of dQ^T(i) into registers and frees its TMEM columns at
 //     once, then adds it into the fp32 accumulator with TMA bulk reductions
 //     (cp.reduce.async.bulk .add.f32) from a 32 KB staging buffer. At the end of a unit it also
 //     reads dV and dK out of TMEM (freeing them for the next unit's first products) and stores
 //     them through the same staging buffer.
 //   * Q tiles with their per-row terms (-lse log2e and D) travel in a 2-stage TMA ring; dO has a
-//     single slot, refilled after dP(i), its last reader, and needed again by dV(i+1) three
+//     single slot, refilled after dV(i), its last reader, and needed again by dP(i+1) three
 //     products later. That single slot is what pays for the staging buffer. K and V of the
 //     next unit load once the current unit's last product has completed.
 //
@@ -569,23 +571,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_dq();
             umma_commit(bar(L::bDQFull));
           }
-          if (i < n_i) {
-            if (!(ok = mbar_wait(bar(L::bOFull), gi & 1, abort_flag, lim) &&
-                       mbar_wait(bar(L::bPDone), gi & 1, abort_flag, lim)))
+          // dP(i) needs dO(i) and its TMEM columns back from the drain; dV(i) needs P^T(i), and
+          // the unit's first dV also the previous unit's dV, dK read out of TMEM. Neither waits
+          // for the other.
+          const bool need_acc = i == 0 && uc > 0;
+          if (i < n_i && D == 64) {
+            // short products: whichever is ready first goes first (dV(i) then covers the drain
+            // of dQ(i-1) when P^T(i) is ready before it)
+            bool dp_done = false, dv_done = false;
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t it = 0; !(dp_done && dv_done); ++it) {
+              if (!dp_done && mbar_test(bar(L::bOFull), gi & 1) &&
+                  (gi == 0 || mbar_test(bar(L::bDQFree), (gi - 1) & 1))) {
+                tc_fence_after();
+                mma_dp();
+                umma_commit(bar(L::bDPFull));
+                dp_done = true;
+              }
+              if (!dv_done && mbar_test(bar(L::bPDone), gi & 1) &&
+                  (!need_acc || mbar_test(bar(L::bAccFree), (uc - 1) & 1))) {
+                tc_fence_after();
+                mma_dv(i > 0);
+                dv_done = true;
+              }
+              if (!(dp_done && dv_done)) {
+                __nanosleep(32);
+                if ((it & 63u) == 63u && (*abort_flag || globaltimer_ns() - t0 > lim)) {
+                  ok = false;
+                  break;
+                }
+              }
+            }
+            if (!ok) break;
+            umma_commit(bar(L::bOEmpty));  // dO(i)'s readers, dP(i) and dV(i), have completed
+          } else if (i < n_i) {
+            // long products: dP(i) first, so that the elementwise warps find it complete when
+            // they finish P^T(i)
+            if (!(ok = mbar_wait(bar(L::bOFull), gi & 1, abort_flag, lim))) break;
+            if (gi > 0 && !(ok = mbar_wait(bar(L::bDQFree), (gi - 1) & 1, abort_flag, lim)))
               break;
-            // the unit's first dV overwrites TMEM the previous unit's epilogue reads
-            if (i == 0 && uc > 0 &&
-                !(ok = mbar_wait(bar(L::bAccFree), (uc - 1) & 1, abort_flag, lim)))
+            tc_fence_after();
+            mma_dp();
+            umma_commit(bar(L::bDPFull));
+            if (!(ok = mbar_wait(bar(L::bPDone), gi & 1, abort_flag, lim))) break;
+            if (need_acc && !(ok = mbar_wait(bar(L::bAccFree), (uc - 1) & 1, abort_flag, lim)))
               break;
             tc_fence_after();
             mma_dv(i > 0);
-            if (gi > 0) {
-              if (!(ok = mbar_wait(bar(L::bDQFree), (gi - 1) & 1, abort_flag, lim))) break;
-              tc_fence_after();
-            }
-            mma_dp();
-            umma_commit(bar(L::bDPFull));
-            umma_commit(bar(L::bOEmpty));
+            umma_commit(bar(L::bOEmpty));  // dV(i) is dO(i)'s last reader
           }
         }
         if (!ok) break;
@@ -637,7 +670,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             skipped = gi;
           }
           issued_q = gi + 1;
-          // dO(i): the single slot frees after dP of the previous tile
+          // dO(i): the single slot frees after dV of the previous tile
           if (gi > 0 && !mbar_wait(bar(L::bOEmpty), (gi - 1) & 1, abort_flag)) {
             ok = false;
             break;
