@@ -571,9 +571,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_dq();
             umma_commit(bar(L::bDQFull));
           }
-          // dP(i) needs dO(i) and its TMEM columns back from the drain; dV(i) needs P^T(i), and
-          // the unit's first dV also the previous unit's dV, dK read out of TMEM. Neither waits
-          // for the other.
+          // dP(i) needs dO(i) and its TMEM columns back from the drain; dV(i) needs dO(i) and
+          // P^T(i), and the unit's first dV also the previous unit's dV, dK read out of TMEM.
+          // Neither waits for the other.
           const bool need_acc = i == 0 && uc > 0;
           if (i < n_i && D == 64) {
             // short products: whichever is ready first goes first (dV(i) then covers the drain
@@ -588,7 +588,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 umma_commit(bar(L::bDPFull));
                 dp_done = true;
               }
-              if (!dv_done && mbar_test(bar(L::bPDone), gi & 1) &&
+              if (!dv_done && mbar_test(bar(L::bOFull), gi & 1) &&
+                  mbar_test(bar(L::bPDone), gi & 1) &&
                   (!need_acc || mbar_test(bar(L::bAccFree), (uc - 1) & 1))) {
                 tc_fence_after();
                 mma_dv(i > 0);
