@@ -113,10 +113,11 @@ struct DeviceState {
   // cudaFuncSetAttribute done for [d == 128][causal][dropout] (atomic: calls from several host
   // threads may launch concurrently; setting an attribute twice is harmless)
   std::atomic<bool> fwd_attr[2][2][2] = {};
+  std::atomic<bool> fwd96_attr[2] = {};  // [causal]: d = 96 without dropout
   std::atomic<bool> fp8_attr[2] = {};  // [causal]
   std::atomic<bool> d256_attr[2] = {};  // [causal]
   std::atomic<bool> bwd_attr[2][2][2] = {};
-  std::atomic<bool> bwd128_attr[4] = {};  // [2 (d = 128) + causal]
+  std::atomic<bool> bwd128_attr[6] = {};  // [2 (d = 128) or 4 (d = 96) + causal]
   std::atomic<bool> bwd256_attr[2] = {};  // [causal]
   int n_sm = 0;  // multiprocessors (grid of the persistent kernels)
 };
@@ -278,12 +279,12 @@ fa_status apply_dropout(Shape& s, const fa_dropout* d) {
   return FA_OK;
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, int DM = D>
 fa_status launch_fwd(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
                      float* lse, const Shape& s, cudaStream_t stream) {
   using L = fa::FwdLayout<D>;
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL, DROPOUT>;
-  std::atomic<bool>& attr = ds->fwd_attr[D == 128][CAUSAL][DROPOUT];
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, DROPOUT, DM>;
+  std::atomic<bool>& attr = DM == 96 ? ds->fwd96_attr[CAUSAL] : ds->fwd_attr[D == 128][CAUSAL][DROPOUT];
   if (!attr) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -442,13 +443,13 @@ fa_status launch_bwd(DeviceState* ds, const void* q, const void* k, const void* 
 
 // Backward at d = 64 and d = 128 (and 96) without dropout: the 128-row query tile kernel
 // (fa_bwd_q128.cuh), between the same preprocess and dQ conversion as launch_bwd.
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int DM = D>
 fa_status launch_bwd_q128(DeviceState* ds, const void* q, const void* k, const void* v,
                           const void* o, const void* dO, const float* lse, void* dq, void* dk,
                           void* dv, void* workspace, const Shape& s, cudaStream_t stream) {
   using L = fa::Bwd128Layout<D>;
-  auto kern = fa::fa_bwd_main_q128<D, CAUSAL>;
-  std::atomic<bool>& attr = ds->bwd128_attr[(D == 128 ? 2 : 0) + CAUSAL];
+  auto kern = fa::fa_bwd_main_q128<D, CAUSAL, DM>;
+  std::atomic<bool>& attr = ds->bwd128_attr[(D == 128 ? (DM == 96 ? 4 : 2) : 0) + CAUSAL];
   if (!attr) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
@@ -673,6 +674,10 @@ fa_status launch_bwd_d256(DeviceState* ds, const void* q, const void* k, const v
 template <int D, bool CAUSAL>
 fa_status fwd_dispatch_d(DeviceState* ds, const void* q, const void* k, const void* v, void* o,
                          float* lse, const Shape& s, cudaStream_t stream) {
+  if constexpr (D == 128) {
+    // d = 96 without dropout on the d = 128 layout, its products over 96 columns
+    if (s.d == 96 && !s.dropout) return launch_fwd<128, CAUSAL, false, 96>(ds, q, k, v, o, lse, s, stream);
+  }
   return s.dropout ? launch_fwd<D, CAUSAL, true>(ds, q, k, v, o, lse, s, stream)
                    : launch_fwd<D, CAUSAL, false>(ds, q, k, v, o, lse, s, stream);
 }
@@ -745,6 +750,12 @@ fa_status bwd_dispatch_d(DeviceState* ds, const void* q, const void* k, const vo
                          void* dv, void* workspace, const Shape& s, cudaStream_t stream) {
   if (s.dropout)
     return launch_bwd<D, CAUSAL, true>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
+  if constexpr (D == 128) {
+    // d = 96 on the d = 128 layout, its products over 96 columns
+    if (s.d == 96)
+      return launch_bwd_q128<128, CAUSAL, 96>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s,
+                                              stream);
+  }
   return launch_bwd_q128<D, CAUSAL>(ds, q, k, v, o, dO, lse, dq, dk, dv, workspace, s, stream);
 }
 
@@ -970,7 +981,7 @@ struct NoAllocDevice {
   void* scratch = nullptr;  // device address of g_noalloc_scratch on this device
   int* status = nullptr;    // device address of g_noalloc_status on this device
   bool bwd_attr[2][2][2] = {};
-  bool bwd128_attr[4] = {};
+  bool bwd128_attr[6] = {};
   int n_sm = 0;
   bool bwd256_attr[2] = {};
 };
@@ -1161,7 +1172,7 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
     local.checked = local.is_sm100 = true;
     local.n_sm = nd.n_sm;
     copy_flags(local.bwd_attr, nd.bwd_attr);
-    for (int c = 0; c < 4; ++c) local.bwd128_attr[c].store(nd.bwd128_attr[c]);
+    for (int c = 0; c < 6; ++c) local.bwd128_attr[c].store(nd.bwd128_attr[c]);
     for (int c = 0; c < 2; ++c) local.bwd256_attr[c].store(nd.bwd256_attr[c]);
   }
   // The first kernel of the backward rewrites every scratch byte the later ones read (dQ
@@ -1172,7 +1183,7 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   {
     std::lock_guard<std::mutex> lock(g_mu);
     copy_flags(g_noalloc[dev].bwd_attr, local.bwd_attr);
-    for (int c = 0; c < 4; ++c) g_noalloc[dev].bwd128_attr[c] = local.bwd128_attr[c].load();
+    for (int c = 0; c < 6; ++c) g_noalloc[dev].bwd128_attr[c] = local.bwd128_attr[c].load();
     for (int c = 0; c < 2; ++c) g_noalloc[dev].bwd256_attr[c] = local.bwd256_attr[c].load();
   }
   return st;

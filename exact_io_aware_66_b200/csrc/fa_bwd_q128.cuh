@@ -126,7 +126,10 @@ __device__ __forceinline__ Bwd128Unit bwd128_unit(int u, const BwdParams& p) {
   return w;
 }
 
-template <int D, bool CAUSAL>
+// D: the shared-memory and TMEM layout (64 or 128 columns of d). DM: the head dimension the
+// products run over (D, or 96 with the d = 128 layout; the tensor maps zero-fill columns past d,
+// so a 96-column contraction over them is exact).
+template <int D, bool CAUSAL, int DM = D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_q128(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
@@ -415,7 +418,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (lane == 0) bulk_wait_group_read0();
       __syncwarp();
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
+      for (int c = 0; c < DM; c += 32) {
         uint32_t v[32];
         if (has) {
           tmem_ld_32x32b_x32(tmem + L::tDV + c + lane_off, v);
@@ -435,9 +438,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
         }
       }
-      uint32_t dk[D / 2];
+      uint32_t dk[DM / 2];
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
+      for (int c = 0; c < DM; c += 32) {
         uint32_t v[32];
         if (has) {
           tmem_ld_32x32b_x32(tmem + L::tDK + c + lane_off, v);
@@ -472,7 +475,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         __syncwarp();
       }
 #pragma unroll
-      for (int chunk = 0; chunk < D / 8; ++chunk)
+      for (int chunk = 0; chunk < DM / 8; ++chunk)
         *reinterpret_cast<uint4*>(stageb + kDKOff + (chunk >> 3) * 4096 +
                                   sw128_offset(lane, chunk & 7)) =
             make_uint4(dk[4 * chunk], dk[4 * chunk + 1], dk[4 * chunk + 2], dk[4 * chunk + 3]);
@@ -492,7 +495,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (warp == 12 && lane == 0) {
       // ------------------------------------------------------------------- MMA ----------
       const uint32_t id_s = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
-      const uint32_t id_acc = idesc_bf16_f32(128, D, false, true);   // dV, dK
+      const uint32_t id_acc = idesc_bf16_f32(128, DM, false, true);  // dV, dK
       const uint32_t id_dq = idesc_bf16_f32(128, D, true, true);     // dQ^T (d = 128), dQ (64)
       const uint64_t dK_k = sdesc_sw128(sbase + L::kK, 16, 1024);          // K, K-major
       const uint64_t dV_k = sdesc_sw128(sbase + L::kV, 16, 1024);          // V, K-major
@@ -508,13 +511,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       auto mma_s = [&](int st) {  // S^T = K Q^T, Q from stage st
         const uint32_t so = static_cast<uint32_t>(st) * L::kTile;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
+        for (int kk = 0; kk < DM / 16; ++kk)
           umma_ss(tmem + L::tS, sdesc_advance(dK_k, kmaj(kk)), sdesc_advance(dQ_k, so + kmaj(kk)),
                   id_s, kk > 0 ? 1u : 0u);
       };
       auto mma_dp = [&]() {  // dP^T = V dO^T
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
+        for (int kk = 0; kk < DM / 16; ++kk)
           umma_ss(tmem + L::tDP, sdesc_advance(dV_k, kmaj(kk)), sdesc_advance(dDO_k, kmaj(kk)),
                   id_s, kk > 0 ? 1u : 0u);
       };

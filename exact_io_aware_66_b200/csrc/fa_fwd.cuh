@@ -177,7 +177,10 @@ __device__ __forceinline__ void fail(int* status, volatile int* abort_flag, int 
   atomicExch(status, code);
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+// D: the shared-memory and TMEM layout (64 or 128 columns of d). DM: the head dimension the
+// products run over (D, or 96 with the d = 128 layout; the tensor maps zero-fill columns past d,
+// so a 96-column contraction over them is exact).
+template <int D, bool CAUSAL, bool DROPOUT, int DM = D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -389,7 +392,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
           const uint32_t tO = tmem + 256 + t * D + (static_cast<uint32_t>((warp & 3) * 32) << 16);
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
+          for (int c = 0; c < DM; c += 32) {
             uint32_t o[32];
             tmem_ld_32x32b_x32(tO + c, o);
             tmem_ld_wait();
@@ -462,11 +465,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int c = 64 * b; c < 64 * b + 64; c += 32) {
             uint32_t o[32];
-            if (n > 0) {
+            if (n > 0 && c < DM) {
               tmem_ld_32x32b_x32(tO + c, o);
               tmem_ld_wait();
               reg_fence(o);
-            } else {  // no PV ever wrote this O accumulator
+            } else {  // no PV ever wrote these O columns (past d, which the store clips)
 #pragma unroll
               for (int i = 0; i < 32; ++i) o[i] = 0u;
             }
@@ -500,7 +503,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (warp == 12 && lane == 0) {
       // ------------------------------------------------------------------ MMA -------------
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, DM, false, true);
       // Operand descriptors are built once; per k-step they are advanced by constant offsets.
       const uint64_t desc_q0 = sdesc_sw128(sbase + L::kQ, 16, 1024);             // K-major
       const uint64_t desc_k0 = sdesc_sw128(sbase + L::kKV, 16, 1024);            // K-major
@@ -514,7 +517,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint64_t b0 = sdesc_advance(desc_k0, (tt % ST) * L::kTileBytes);
         const uint32_t d = tmem + t * 128;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < DM / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
           umma_ss(d, sdesc_advance(a0, off), sdesc_advance(b0, off), idesc_qk, kk > 0 ? 1u : 0u);
         }
