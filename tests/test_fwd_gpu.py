@@ -50,11 +50,13 @@ def test_fwd_first_config_full():
     assert_fwd_ok(err, w.name)
 
 
-@pytest.mark.parametrize("name", ["causal_train_b1h16n16384d128", "causal_fwd_b1h8n131072d128"])
+@pytest.mark.parametrize("name", ["causal_train_b1h16n16384d128", "causal_fwd_b1h8n131072d128",
+                                  "causal_train_b4h16n4096d96"])
 def test_fwd_full_size_sampled_rows(name):
-    """The two long-sequence workloads, same launch configuration as the bench: sampled query
-    rows (512, or 256 at N = 131072) against the oracle, and every output finite. (The N = 2048
-    and N = 4096 workloads are compared element by element in test_bwd_gpu.py.)"""
+    """The two long-sequence workloads and the d = 96 one (its products run over 96 columns of
+    the d = 128 layout), same launch configuration as the bench: sampled query rows (512, or 256)
+    against the oracle, and every output finite. (The d = 64 N = 2048 and d = 128 N = 4096
+    workloads are compared element by element in test_bwd_gpu.py.)"""
     w = WORKLOADS[name]
     x = workload_inputs(w, with_do=False)
     o, lse = _run(x, w.causal)
